@@ -1,0 +1,376 @@
+// libsala C-ABI host layer: argument validation, workspace layout, launches.
+//
+// Every entry point validates its arguments before launching anything and
+// returns SALA_ERR_INVALID_ARG / SALA_ERR_UNSUPPORTED / SALA_ERR_WORKSPACE
+// synchronously; launches go to the caller's stream.  The library allocates
+// no memory: scratch lives in the caller's workspace.
+#include <algorithm>
+#include <math.h>
+#include <string.h>
+
+#include "../../include/sala.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "linear_simt.cuh"
+#include "prologue.cuh"
+#include "select.cuh"
+#include "sparse_simt.cuh"
+
+using namespace sala;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+inline bool aligned16_or_null(const void* p) { return !p || ((uintptr_t)p & 15u) == 0; }
+
+inline size_t elt_size(sala_dtype t) { return t == SALA_F32 ? 4 : 2; }
+
+inline sala_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SALA_OK : SALA_ERR_CUDA;
+}
+
+template <typename K>
+inline cudaError_t allow_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+sala_status check_linear(const sala_linear_desc* d) {
+  if (!d) return SALA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->seqlen < 1 || d->heads < 1 || d->chunk < 1) return SALA_ERR_INVALID_ARG;
+  if (d->dtype != SALA_F32 && d->dtype != SALA_BF16) return SALA_ERR_INVALID_ARG;
+  if (!(d->rms_eps >= 0.f) || !(d->rope_base > 0.f) || !isfinite(d->scale) || d->pos0 < 0)
+    return SALA_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return SALA_ERR_UNSUPPORTED;
+  if (d->seqlen % d->chunk != 0 || d->seqlen % kSimtChunk != 0) return SALA_ERR_UNSUPPORTED;
+  return SALA_OK;
+}
+
+sala_status check_sparse(const sala_sparse_desc* d) {
+  if (!d) return SALA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->seqlen < 1 || d->q_heads < 1 || d->kv_heads < 1) return SALA_ERR_INVALID_ARG;
+  if (d->q_heads % d->kv_heads != 0) return SALA_ERR_INVALID_ARG;
+  if (d->topk < 0 || d->n_init < 0 || d->n_local < 1 || d->block < 1) return SALA_ERR_INVALID_ARG;
+  if (d->dtype != SALA_F32 && d->dtype != SALA_BF16) return SALA_ERR_INVALID_ARG;
+  if (!(d->rms_eps >= 0.f) || !isfinite(d->scale)) return SALA_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return SALA_ERR_UNSUPPORTED;
+  if (d->block != 64 || d->seqlen % d->block != 0) return SALA_ERR_UNSUPPORTED;
+  if (d->topk + d->n_init + d->n_local > 1024) return SALA_ERR_UNSUPPORTED;
+  if (d->seqlen / d->block > 49152) return SALA_ERR_UNSUPPORTED;   // select smem: 4 B per block
+  return SALA_OK;
+}
+
+inline float sparse_scale(const sala_sparse_desc* d) {
+  return d->scale > 0.f ? d->scale : 1.0f / sqrtf((float)d->head_dim);
+}
+
+struct LinearWs {
+  size_t qn, kn, total;
+};
+LinearWs linear_ws(const sala_linear_desc* d) {
+  const size_t n = (size_t)d->batch * d->seqlen * d->heads * d->head_dim;
+  LinearWs w;
+  w.qn = 0;
+  w.kn = align_up(n * 2);
+  w.total = w.kn + align_up(n * 2);
+  return w;
+}
+
+template <typename T, int D>
+sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, const void* v,
+                       const void* gate, const float* lambda, const float* wq, const float* wk,
+                       const float* state_in, float* state_out, void* out, char* ws,
+                       cudaStream_t st) {
+  const LinearWs w = linear_ws(d);
+  auto* qn = reinterpret_cast<__nv_bfloat16*>(ws + w.qn);
+  auto* kn = reinterpret_cast<__nv_bfloat16*>(ws + w.kn);
+  const long long tokens = (long long)d->batch * d->seqlen;
+  const int pro_blocks = (int)((tokens + kRopeTokens - 1) / kRopeTokens);
+  linear_prologue_kernel<T, D><<<pro_blocks, kPrologueThreads, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), wq, wk, qn, kn, tokens, d->seqlen,
+      d->heads, d->pos0, log2((double)d->rope_base), d->rms_eps);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  const size_t smem = sizeof(SimtSmem<D>);
+  if (allow_smem(linear_chunk_simt_kernel<T, D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  const int grid = d->batch * d->heads * (D / kSimtCols);
+  linear_chunk_simt_kernel<T, D><<<grid, kSimtThreads, smem, st>>>(
+      qn, kn, static_cast<const T*>(v), static_cast<const T*>(gate), lambda, state_in, state_out,
+      static_cast<T*>(out), d->seqlen, d->heads, d->scale);
+  return launch_status();
+}
+
+template <typename T, int D>
+sala_status run_select(const sala_sparse_desc* d, const void* q, const void* k, const float* wq,
+                       const float* wk, void* q_norm, void* k_norm, float* kbar, int32_t* idx,
+                       char* ws, cudaStream_t st) {
+  const int nb = d->seqlen / d->block;
+  float* qsum = reinterpret_cast<float*>(ws);
+  sparse_prologue_kernel<T, D><<<d->batch * nb * d->kv_heads, kPrologueThreads, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), wq, wk,
+      static_cast<__nv_bfloat16*>(q_norm), static_cast<__nv_bfloat16*>(k_norm), qsum, kbar,
+      d->seqlen, d->q_heads, d->kv_heads, d->block, d->rms_eps);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  const size_t smem = (size_t)nb * sizeof(uint32_t);
+  if (allow_smem(select_topk_kernel<D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  const int width = d->topk + d->n_init + d->n_local;
+  select_topk_kernel<D><<<d->batch * d->kv_heads * nb, kSelectThreads, smem, st>>>(
+      qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width);
+  return launch_status();
+}
+
+template <typename T, int D>
+sala_status run_sparse_prefill(const sala_sparse_desc* d, const void* qn, const void* kn,
+                               const void* v, const void* gate, const int32_t* idx, void* out,
+                               cudaStream_t st) {
+  const int nb = d->seqlen / d->block;
+  const size_t smem = sizeof(SpSimtSmem<D>);
+  if (allow_smem(sparse_attn_simt_kernel<T, D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  sparse_attn_simt_kernel<T, D><<<d->batch * nb * d->kv_heads, kSpSimtThreads, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(qn), static_cast<const __nv_bfloat16*>(kn),
+      static_cast<const T*>(v), static_cast<const T*>(gate), idx, static_cast<T*>(out),
+      d->seqlen, d->q_heads, d->kv_heads, d->topk + d->n_init + d->n_local, sparse_scale(d));
+  return launch_status();
+}
+
+struct DecodeWs {
+  size_t qhat, qgrp, keys, idx, part, total;
+};
+DecodeWs decode_ws(const sala_decode_desc* d) {
+  const sala_sparse_desc& s = d->sp;
+  const size_t B = s.batch, Hq = s.q_heads, Hkv = s.kv_heads, D = s.head_dim;
+  const size_t width = s.topk + s.n_init + s.n_local;
+  const size_t capb = (size_t)(d->cache_capacity / s.block);
+  DecodeWs w;
+  w.qhat = 0;
+  w.qgrp = w.qhat + align_up(B * Hq * D * 4);
+  w.keys = w.qgrp + align_up(B * Hkv * D * 4);
+  w.idx = w.keys + align_up(B * Hkv * capb * 4);
+  w.part = w.idx + align_up(B * Hkv * width * 4);
+  w.total = w.part + align_up(B * Hkv * width * (Hq / Hkv) * (D + 2) * 4);
+  return w;
+}
+
+sala_status check_decode(const sala_decode_desc* d) {
+  if (!d) return SALA_ERR_INVALID_ARG;
+  if (d->n_linear < 1 || d->n_linear > SALA_MAX_LAYERS - 1) return SALA_ERR_INVALID_ARG;
+  sala_linear_desc l = d->lin;
+  l.seqlen = l.chunk = 64;
+  l.pos0 = 0;
+  sala_status s = check_linear(&l);
+  if (s != SALA_OK) return s;
+  sala_sparse_desc sp = d->sp;
+  sp.seqlen = sp.block;
+  s = check_sparse(&sp);
+  if (s != SALA_OK) return s;
+  if (d->lin.batch != d->sp.batch || d->lin.dtype != d->sp.dtype) return SALA_ERR_INVALID_ARG;
+  if (d->cache_capacity < d->sp.block || d->cache_capacity % d->sp.block != 0) return SALA_ERR_INVALID_ARG;
+  if (d->cache_capacity / d->sp.block > 49152) return SALA_ERR_UNSUPPORTED;
+  return SALA_OK;
+}
+
+template <typename T, int DL, int DS>
+sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void* k_cache,
+                       void* v_cache, float* kbar, float* ksum, int64_t cur_len, char* ws,
+                       cudaStream_t st) {
+  const sala_linear_desc& L = d->lin;
+  DecodeLinearArgs a;
+  memset(&a, 0, sizeof(a));
+  for (int l = 0; l < d->n_linear; ++l) {
+    a.q[l] = io->q[l]; a.k[l] = io->k[l]; a.v[l] = io->v[l]; a.gate[l] = io->gate[l];
+    a.wq[l] = io->wq[l]; a.wk[l] = io->wk[l]; a.lambda[l] = io->lambda[l];
+    a.state[l] = io->lin_state[l]; a.out[l] = io->out[l];
+  }
+  decode_linear_kernel<T, DL><<<d->n_linear * L.batch * L.heads * (DL / 64), 256, 0, st>>>(
+      a, L.batch, L.heads, cur_len, log2((double)L.rope_base), L.rms_eps, L.scale);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+
+  const sala_sparse_desc& S = d->sp;
+  const int sl = d->n_linear;
+  const DecodeWs w = decode_ws(d);
+  float* qhat = reinterpret_cast<float*>(ws + w.qhat);
+  float* qgrp = reinterpret_cast<float*>(ws + w.qgrp);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ws + w.keys);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  float* part = reinterpret_cast<float*>(ws + w.part);
+  const long long capb = d->cache_capacity / S.block;
+  const int width = S.topk + S.n_init + S.n_local;
+  decode_sparse_prep_kernel<T, DS><<<S.batch, 256, 0, st>>>(
+      static_cast<const T*>(io->q[sl]), static_cast<const T*>(io->k[sl]),
+      static_cast<const T*>(io->v[sl]), io->wq[sl], io->wk[sl],
+      static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), kbar, ksum,
+      qhat, qgrp, S.q_heads, S.kv_heads, d->cache_capacity, cur_len, S.block, S.rms_eps);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  const int bcur = (int)(cur_len / S.block);
+  const int n_cand = std::max(0, bcur - S.n_local + 1 - S.n_init);
+  if (n_cand > S.topk) {
+    const long long total = (long long)S.batch * S.kv_heads * n_cand;
+    decode_scores_kernel<DS><<<(unsigned)((total + 7) / 8), 256, 0, st>>>(
+        qgrp, kbar, keys, S.kv_heads, capb, S.n_init, n_cand, total);
+    if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  }
+  const size_t smem = (size_t)std::max(n_cand, 1) * 4;
+  if (allow_smem(decode_topk_kernel, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  decode_topk_kernel<<<S.batch * S.kv_heads, kSelectThreads, smem, st>>>(
+      keys, idx, S.kv_heads, capb, bcur, S.topk, S.n_init, S.n_local, width);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  const size_t asmem = sizeof(float) * 64 * (2 * DS + 1);
+  if (allow_smem(decode_attn_kernel<DS>, asmem) != cudaSuccess) return SALA_ERR_CUDA;
+  decode_attn_kernel<DS><<<S.batch * S.kv_heads * width, 256, asmem, st>>>(
+      qhat, static_cast<const __nv_bfloat16*>(k_cache), static_cast<const __nv_bfloat16*>(v_cache),
+      idx, part, S.q_heads, S.kv_heads, d->cache_capacity, cur_len, S.block, width,
+      sparse_scale(&S));
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  decode_combine_kernel<T, DS><<<S.batch * S.q_heads, DS, 0, st>>>(
+      part, static_cast<const T*>(io->gate[sl]), static_cast<T*>(io->out[sl]), S.q_heads,
+      S.kv_heads, width);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int sala_sparse_index_width(const sala_sparse_desc* d) {
+  return d ? d->topk + d->n_init + d->n_local : -1;
+}
+
+size_t sala_linear_workspace_size(const sala_linear_desc* d) {
+  if (check_linear(d) != SALA_OK) return 0;
+  return linear_ws(d).total;
+}
+
+sala_status sala_linear_prefill(const sala_linear_desc* d, const void* q, const void* k,
+                                const void* v, const void* gate, const float* lambda,
+                                const float* wq, const float* wk, const float* state_in,
+                                float* state_out, void* out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  sala_status s = check_linear(d);
+  if (s != SALA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(out) ||
+      !aligned16(lambda) || !aligned16(wq) || !aligned16(wk) || !aligned16_or_null(state_in) ||
+      !aligned16_or_null(state_out))
+    return SALA_ERR_INVALID_ARG;
+  if (ws_bytes < linear_ws(d).total || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (d->dtype == SALA_BF16) {
+    if (d->head_dim == 128)
+      return run_linear<__nv_bfloat16, 128>(d, q, k, v, gate, lambda, wq, wk, state_in, state_out, out, ws, st);
+    return run_linear<__nv_bfloat16, 64>(d, q, k, v, gate, lambda, wq, wk, state_in, state_out, out, ws, st);
+  }
+  if (d->head_dim == 128)
+    return run_linear<float, 128>(d, q, k, v, gate, lambda, wq, wk, state_in, state_out, out, ws, st);
+  return run_linear<float, 64>(d, q, k, v, gate, lambda, wq, wk, state_in, state_out, out, ws, st);
+}
+
+size_t sala_sparse_workspace_size(const sala_sparse_desc* d) {
+  if (check_sparse(d) != SALA_OK) return 0;
+  return align_up((size_t)d->batch * (d->seqlen / d->block) * d->kv_heads * d->head_dim * 4);
+}
+
+sala_status sala_sparse_select(const sala_sparse_desc* d, const void* q, const void* k,
+                               const float* wq, const float* wk, void* q_norm, void* k_norm,
+                               float* kbar, int32_t* idx, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  sala_status s = check_sparse(d);
+  if (s != SALA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(wq) || !aligned16(wk) || !aligned16(q_norm) ||
+      !aligned16(k_norm) || !aligned16(kbar) || !aligned16(idx))
+    return SALA_ERR_INVALID_ARG;
+  if (ws_bytes < sala_sparse_workspace_size(d) || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (d->dtype == SALA_BF16) {
+    if (d->head_dim == 128)
+      return run_select<__nv_bfloat16, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+    return run_select<__nv_bfloat16, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+  }
+  if (d->head_dim == 128)
+    return run_select<float, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+  return run_select<float, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+}
+
+sala_status sala_sparse_prefill(const sala_sparse_desc* d, const void* q_norm,
+                                const void* k_norm, const void* v, const void* gate,
+                                const int32_t* idx, void* out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  sala_status s = check_sparse(d);
+  if (s != SALA_OK) return s;
+  if (!aligned16(q_norm) || !aligned16(k_norm) || !aligned16(v) || !aligned16(gate) ||
+      !aligned16(idx) || !aligned16(out))
+    return SALA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == SALA_BF16) {
+    if (d->head_dim == 128)
+      return run_sparse_prefill<__nv_bfloat16, 128>(d, q_norm, k_norm, v, gate, idx, out, st);
+    return run_sparse_prefill<__nv_bfloat16, 64>(d, q_norm, k_norm, v, gate, idx, out, st);
+  }
+  if (d->head_dim == 128)
+    return run_sparse_prefill<float, 128>(d, q_norm, k_norm, v, gate, idx, out, st);
+  return run_sparse_prefill<float, 64>(d, q_norm, k_norm, v, gate, idx, out, st);
+}
+
+size_t sala_decode_workspace_size(const sala_decode_desc* d) {
+  if (check_decode(d) != SALA_OK) return 0;
+  return decode_ws(d).total;
+}
+
+sala_status sala_decode_step(const sala_decode_desc* d, const sala_decode_io* io, void* k_cache,
+                             void* v_cache, float* kbar, float* ksum, int64_t cur_len,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  sala_status s = check_decode(d);
+  if (s != SALA_OK) return s;
+  if (!io || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kbar) || !aligned16(ksum))
+    return SALA_ERR_INVALID_ARG;
+  if (cur_len < 0 || cur_len >= d->cache_capacity) return SALA_ERR_INVALID_ARG;
+  for (int l = 0; l <= d->n_linear; ++l) {
+    if (!aligned16(io->q[l]) || !aligned16(io->k[l]) || !aligned16(io->v[l]) ||
+        !aligned16(io->gate[l]) || !aligned16(io->out[l]) || !aligned16(io->wq[l]) ||
+        !aligned16(io->wk[l]))
+      return SALA_ERR_INVALID_ARG;
+    if (l < d->n_linear && (!aligned16(io->lambda[l]) || !aligned16(io->lin_state[l])))
+      return SALA_ERR_INVALID_ARG;
+  }
+  if (ws_bytes < decode_ws(d).total || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const int dl = d->lin.head_dim, ds = d->sp.head_dim;
+  if (dl != ds) return SALA_ERR_UNSUPPORTED;
+  if (d->lin.dtype == SALA_BF16) {
+    if (dl == 128) return run_decode<__nv_bfloat16, 128, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+    return run_decode<__nv_bfloat16, 64, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+  }
+  if (dl == 128) return run_decode<float, 128, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+  return run_decode<float, 64, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+}
+
+const char* sala_status_string(sala_status s) {
+  switch (s) {
+    case SALA_OK: return "ok";
+    case SALA_ERR_INVALID_ARG: return "invalid argument";
+    case SALA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case SALA_ERR_CUDA: return "CUDA error";
+    case SALA_ERR_TIMEOUT: return "device wait timed out";
+    case SALA_ERR_WORKSPACE: return "workspace too small";
+    case SALA_ERR_DEVICE_FAULT: return "device bounds check failed";
+  }
+  return "unknown status";
+}
+
+sala_status sala_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SALA_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return SALA_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SALA_ERR_CUDA;
+  if (v & kStatusTimeout) return SALA_ERR_TIMEOUT;
+  if (v & kStatusBounds) return SALA_ERR_DEVICE_FAULT;
+  return SALA_OK;
+}
+
+int sala_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+// Block scoring and top-k selection of the sparse layer.
+//
+// InfLLM-V2-style selection (acgfav.com "SALA 混合架构": a fine-grained block
+// selection lets each query attend to only a small set of key blocks).
+// Query block i of kv head g scores each causal candidate block
+// j in [n_init, i - n_local] by <qsum_i^g, kbar_j^g> / sqrt(d), where qsum is
+// the sum over the group's q heads of the block-mean normalised query and
+// kbar the block-mean normalised key.  It keeps the initial blocks
+// [0, n_init), the local blocks [i-n_local+1, i] and the top-k candidates
+// (ties to the lower block index), written in ascending order, -1 padded.
+//
+// The k-th largest score is found exactly by a 4-pass radix select over the
+// order-preserving uint32 image of the fp32 scores; the selected set is then
+// emitted in index order by a block-wide ordered compaction, so the output is
+// deterministic and matches the tie rule exactly.
+#pragma once
+
+#include "common.cuh"
+
+namespace sala {
+
+constexpr int kSelectThreads = 256;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
+  // scratch: >= kSelectThreads/32 + 1 ints
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kSelectThreads / 32 ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kSelectThreads / 32) scratch[lane] = w;   // inclusive per warp
+  }
+  __syncthreads();
+  const int before = (warp ? scratch[warp - 1] : 0) + x - v;
+  *total = scratch[kSelectThreads / 32 - 1];
+  __syncthreads();
+  return before;
+}
+
+// Top-k of n_cand keys held in shared memory (k < n_cand): writes the chosen
+// candidate numbers c (ascending) to out[0..k) as base + c.  Whole CTA of
+// kSelectThreads threads; hist / scan_scratch / s_prefix / s_need in smem.
+__device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_cand, int k,
+                                                 int32_t* out, int base, int* hist,
+                                                 int* scan_scratch, uint32_t* s_prefix,
+                                                 int* s_need) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int e = tid; e < 256; e += kSelectThreads) hist[e] = 0;
+    __syncthreads();
+    for (int c = tid; c < n_cand; c += kSelectThreads) {
+      const uint32_t key = keys[c];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int cum = 0, bin = 0;
+      for (bin = 255; bin >= 0; --bin) {
+        if (cum + hist[bin] >= need) break;
+        cum += hist[bin];
+      }
+      *s_prefix = prefix | ((uint32_t)bin << shift);
+      *s_need = need - cum;
+    }
+    __syncthreads();
+    prefix = *s_prefix;
+    need = *s_need;
+    mask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;   // key of the k-th largest score; `need` ties at T are taken
+
+  // ordered compaction: each thread owns a contiguous range of candidates
+  const int per = (n_cand + kSelectThreads - 1) / kSelectThreads;
+  const int lo = min(n_cand, tid * per), hi = min(n_cand, lo + per);
+  int n_gt = 0, n_eq = 0;
+  for (int c = lo; c < hi; ++c) {
+    const uint32_t key = keys[c];
+    n_gt += key > T;
+    n_eq += key == T;
+  }
+  int tot;
+  const int eq_before = block_exclusive_scan(n_eq, scan_scratch, &tot);
+  const int take_eq = max(0, min(n_eq, need - eq_before));
+  const int out_before = block_exclusive_scan(n_gt + take_eq, scan_scratch, &tot);
+  int pos = out_before, eq_seen = 0;
+  for (int c = lo; c < hi; ++c) {
+    const uint32_t key = keys[c];
+    bool sel = key > T;
+    if (key == T) { sel = eq_seen < take_eq; ++eq_seen; }
+    if (sel) {
+      if (pos < k) out[pos++] = base + c;
+      else set_status(kStatusBounds);
+    }
+  }
+}
+
+// One CTA per (batch, kv head g, query block i).  Dynamic smem: n_b uint32 keys.
+template <int D>
+__global__ void __launch_bounds__(kSelectThreads)
+select_topk_kernel(const float* __restrict__ qsum, const float* __restrict__ kbar,
+                   int32_t* __restrict__ idx, int nb, int Hkv, int topk, int n_init,
+                   int n_local, int width) {
+  extern __shared__ uint32_t keys[];
+  __shared__ float qv[D];
+  __shared__ int hist[256];
+  __shared__ int scan_scratch[kSelectThreads / 32 + 1];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need;
+
+  const int i = blockIdx.x % nb;
+  const int g = (blockIdx.x / nb) % Hkv;
+  const int b = blockIdx.x / (nb * Hkv);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
+
+  const int n_cand = max(0, i - n_local + 1 - n_init);
+  const int k = min(topk, n_cand);
+  // initial blocks
+  const int n_first = min(n_init, i + 1);
+  for (int e = tid; e < n_first; e += kSelectThreads) row[e] = e;
+  const int local_lo = max(n_init, i - n_local + 1);
+  const int n_loc = max(0, i - local_lo + 1);
+  for (int e = tid; e < n_loc; e += kSelectThreads) row[n_first + k + e] = local_lo + e;
+  for (int e = n_first + k + n_loc + tid; e < width; e += kSelectThreads) row[e] = -1;
+  if (k == 0) return;
+  if (k == n_cand) {
+    for (int e = tid; e < n_cand; e += kSelectThreads) row[n_first + e] = n_init + e;
+    return;
+  }
+
+  // scores of the candidates, one warp per candidate row (coalesced over d)
+  for (int e = tid; e < D; e += kSelectThreads) qv[e] = qsum[(((long long)b * nb + i) * Hkv + g) * D + e];
+  __syncthreads();
+  const float inv_sqrt_d = rsqrtf((float)D);
+  for (int c = warp; c < n_cand; c += kSelectThreads / 32) {
+    const float* kr = kbar + (((long long)b * nb + n_init + c) * Hkv + g) * D;
+    float p = 0.f;
+#pragma unroll
+    for (int e = lane; e < D; e += 32) p = fmaf(qv[e], kr[e], p);
+    p = warp_sum(p);
+    if (lane == 0) keys[c] = score_key(p * inv_sqrt_d);
+  }
+  __syncthreads();
+
+  topk_emit_sorted(keys, n_cand, k, row + n_first, n_init, hist, scan_scratch, &s_prefix, &s_need);
+}
+
+}  // namespace sala

@@ -1,0 +1,249 @@
+"""libsala CUDA path against the fp64 oracle on identical seeded inputs (B200)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hybrid_sparse_linear_lightning_b200 import workloads as wl
+from tests.parity import TOL, check_index_rows, f64, lam_tensor, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sala(cuda_device):
+    from hybrid_sparse_linear_lightning_b200 import sala as s
+    return s
+
+
+def _w(name, **kw):
+    import dataclasses
+    w = wl.WORKLOADS[name]
+    lin = kw.pop("linear", None)
+    sp = kw.pop("sparse", None)
+    if lin:
+        w = dataclasses.replace(w, linear=dataclasses.replace(w.linear, **lin))
+    if sp:
+        w = dataclasses.replace(w, sparse=dataclasses.replace(w.sparse, **sp))
+    return dataclasses.replace(w, **kw)
+
+
+# ----------------------------------------------------------------------------- linear layers
+
+def run_linear_case(sala, w, layer=0, state_in=None, pos0=0, heads=None, seqlen=None):
+    dev = torch.device("cuda")
+    q, k, v, g = wl.layer_inputs(w, layer, dev, seqlen=seqlen)
+    lam = lam_tensor(w, dev)
+    wq = wl.rms_weights(w.linear.head_dim, dev)
+    out, st = sala.linear_prefill(q, k, v, g, lam, wq, wq, chunk=w.linear.chunk, pos0=pos0,
+                                  state_in=state_in, want_state=True)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    ref, S = oracle.linear_layer(f64(q), f64(k), f64(v), f64(g), f64(lam), f64(wq), f64(wq),
+                                 chunk=w.linear.chunk, pos0=pos0, state_in=None if state_in is None
+                                 else f64(state_in), heads=heads)
+    return out, st, ref, S
+
+
+def test_linear_tiny_f32(sala):
+    w = wl.WORKLOADS["tiny_2k_f32"]
+    out, st, ref, S = run_linear_case(sala, w)
+    assert out.dtype == torch.float32
+    assert rel_err(f64(out), ref) <= TOL
+    assert rel_err(f64(st), S) <= TOL
+
+
+@pytest.mark.parametrize("lam_kind,seqlen", [("schedule", 4160), ("half_one", 2048)])
+def test_linear_bf16_d128(sala, lam_kind, seqlen):
+    w = _w("group_32k", linear={"lam_kind": lam_kind})
+    out, st, ref, S = run_linear_case(sala, w, seqlen=seqlen)
+    assert rel_err(f64(out), ref) <= TOL
+    assert rel_err(f64(st), S) <= TOL
+
+
+def test_linear_special_lambdas(sala):
+    dev = torch.device("cuda")
+    w = _w("group_32k")
+    q, k, v, g = wl.layer_inputs(w, 1, dev, seqlen=1024)
+    H = w.linear.heads
+    lam = torch.tensor([0.0 if h % 3 == 0 else (1.0 if h % 3 == 1 else 0.5) for h in range(H)],
+                       dtype=torch.float32, device=dev)
+    wq = wl.rms_weights(128, dev)
+    out, _ = sala.linear_prefill(q, k, v, g, lam, wq, wq)
+    ref, _ = oracle.linear_layer(f64(q), f64(k), f64(v), f64(g), f64(lam), f64(wq), f64(wq))
+    assert rel_err(f64(out), ref) <= TOL
+
+
+def test_linear_resume_segments(sala):
+    """Prefill of [0, N) == prefill [0, N/2) then [N/2, N) with pos0 and the carried state."""
+    dev = torch.device("cuda")
+    w = _w("group_32k")
+    q, k, v, g = wl.layer_inputs(w, 2, dev, seqlen=2048)
+    lam = lam_tensor(w, dev)
+    wq = wl.rms_weights(128, dev)
+    full, s_full = sala.linear_prefill(q, k, v, g, lam, wq, wq, want_state=True)
+    h = 1024
+    sl = lambda t, a, b: t[:, a:b].contiguous()
+    o1, s1 = sala.linear_prefill(sl(q, 0, h), sl(k, 0, h), sl(v, 0, h), sl(g, 0, h), lam, wq, wq,
+                                 want_state=True)
+    o2, s2 = sala.linear_prefill(sl(q, h, 2048), sl(k, h, 2048), sl(v, h, 2048), sl(g, h, 2048),
+                                 lam, wq, wq, pos0=h, state_in=s1, want_state=True)
+    ref, S = oracle.linear_layer(f64(q), f64(k), f64(v), f64(g), f64(lam), f64(wq), f64(wq))
+    assert rel_err(f64(torch.cat([o1, o2], 1)), ref) <= TOL
+    assert rel_err(f64(s2), S) <= TOL
+    assert rel_err(f64(full), ref) <= TOL
+
+
+# ----------------------------------------------------------------------------- sparse layer
+
+def run_sparse_case(sala, w, seqlen=None, query_blocks=None):
+    dev = torch.device("cuda")
+    sp = w.sparse
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev, seqlen=seqlen)
+    wq = wl.rms_weights(sp.head_dim, dev)
+    qn, kn, kbar, idx = sala.sparse_select(q, k, wq, wq, block=sp.block, topk=sp.topk,
+                                           n_init=sp.n_init, n_local=sp.n_local)
+    out = sala.sparse_prefill(qn, kn, v, g, idx, block=sp.block, topk=sp.topk, n_init=sp.n_init,
+                              n_local=sp.n_local)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    ref, (qh, kh, kb, ridx, scores) = oracle.sparse_layer(
+        f64(q), f64(k), f64(v), f64(g), f64(wq), f64(wq), block=sp.block, topk=sp.topk,
+        n_init=sp.n_init, n_local=sp.n_local, query_blocks=query_blocks)
+    return dict(q=q, k=k, v=v, g=g, qn=qn, kn=kn, kbar=kbar, idx=idx, out=out, ref=ref, qh=qh,
+                kh=kh, kb=kb, ridx=ridx, scores=scores)
+
+
+def _compare_sparse(r, sp, rows=None):
+    B, N, Hq, D = r["q"].shape
+    nb = N // sp.block
+    rows = list(range(nb)) if rows is None else list(rows)
+    gidx = r["idx"].cpu().numpy()
+    n_tie = check_index_rows(gidx, r["ridx"], r["scores"], sp.topk, sp.n_init, sp.n_local, rows)
+    assert rel_err(f64(r["kbar"]), np.transpose(r["kb"], (0, 2, 1, 3))) <= 1e-5
+    assert rel_err(f64(r["qn"]), r["qh"]) <= TOL
+    assert rel_err(f64(r["kn"]), r["kh"]) <= TOL
+    # outputs of query blocks whose selection matched the oracle's exactly
+    same = np.zeros((B, N, Hq), dtype=bool)
+    G = Hq // sp.kv_heads if hasattr(sp, "kv_heads") else 1
+    for b in range(B):
+        for i in rows:
+            for gg in range(r["k"].shape[2]):
+                if np.array_equal(gidx[b, gg, i], r["ridx"][b, gg, i]):
+                    same[b, i * sp.block:(i + 1) * sp.block, gg * G:(gg + 1) * G] = True
+    mask = np.broadcast_to(same[..., None], r["ref"].shape)
+    assert rel_err(f64(r["out"]), r["ref"], mask) <= TOL
+    return n_tie
+
+
+def test_sparse_tiny_f32(sala):
+    w = wl.WORKLOADS["tiny_2k_f32"]
+    r = run_sparse_case(sala, w)
+    assert r["out"].dtype == torch.float32
+    assert _compare_sparse(r, w.sparse) == 0
+
+
+@pytest.mark.parametrize("seqlen,topk,n_local", [(4160, 16, 2), (8192, 64, 4)])
+def test_sparse_bf16_d128(sala, seqlen, topk, n_local):
+    w = _w("group_32k", sparse={"topk": topk, "n_local": n_local})
+    r = run_sparse_case(sala, w, seqlen=seqlen)
+    _compare_sparse(r, w.sparse)
+
+
+def test_sparse_prefill_given_oracle_indices(sala):
+    """The attention kernel alone, fed the oracle's own selection."""
+    dev = torch.device("cuda")
+    w = _w("group_32k")
+    sp = w.sparse
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev, seqlen=4096)
+    wq = wl.rms_weights(128, dev)
+    qh, kh, _, ridx, _ = oracle.sparse_select(f64(q), f64(k), f64(wq), f64(wq), block=64,
+                                              topk=sp.topk, n_init=sp.n_init, n_local=sp.n_local)
+    qn = torch.from_numpy(qh).to(dev, torch.bfloat16)
+    kn = torch.from_numpy(kh).to(dev, torch.bfloat16)
+    idx = torch.from_numpy(ridx).to(dev)
+    out = sala.sparse_prefill(qn, kn, v, g, idx, topk=sp.topk, n_init=sp.n_init,
+                              n_local=sp.n_local)
+    ref = oracle.sigmoid(f64(g)) * oracle.sparse_attention(qh, kh, f64(v), ridx, 64)
+    assert rel_err(f64(out), ref) <= TOL
+
+
+@pytest.mark.parametrize("case", ["one_block", "topk0", "local_covers_all", "mha", "init3"])
+def test_sparse_edges(sala, case):
+    if case == "one_block":
+        w = _w("group_32k")
+        seqlen = 64
+    elif case == "topk0":
+        w = _w("group_32k", sparse={"topk": 0})
+        seqlen = 1024
+    elif case == "local_covers_all":
+        w = _w("group_32k", sparse={"n_local": 40})
+        seqlen = 2048
+    elif case == "mha":
+        w = _w("tiny_2k_f32", sparse={"kv_heads": 4}, dtype="bf16")
+        seqlen = 1024
+    else:
+        w = _w("group_32k", sparse={"n_init": 3, "topk": 5})
+        seqlen = 1024
+    r = run_sparse_case(sala, w, seqlen=seqlen)
+    _compare_sparse(r, w.sparse)
+
+
+# ----------------------------------------------------------------------------- decode
+
+def test_decode_steps(sala):
+    """Prefill a short group, then decode tokens across a block boundary."""
+    dev = torch.device("cuda")
+    w = _w("group_32k", sparse={"topk": 4, "n_local": 2})
+    N, steps, cap = 640, 70, 1024
+    sp, ln = w.sparse, w.linear
+    B, H, D = 1, ln.heads, ln.head_dim
+    wq = wl.rms_weights(D, dev)
+    lam = lam_tensor(w, dev)
+    states, ref_states, lin_in = [], [], []
+    for l in range(w.n_linear):
+        q, k, v, g = wl.layer_inputs(w, l, dev, seqlen=N)
+        _, st = sala.linear_prefill(q, k, v, g, lam, wq, wq, want_state=True)
+        _, S = oracle.linear_layer(f64(q), f64(k), f64(v), f64(g), f64(lam), f64(wq), f64(wq))
+        states.append(st)
+        ref_states.append(S)
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev, seqlen=N)
+    k_cache = torch.zeros((B, cap, sp.kv_heads, D), dtype=torch.bfloat16, device=dev)
+    v_cache = torch.zeros_like(k_cache)
+    kbar = torch.zeros((B, cap // 64, sp.kv_heads, D), dtype=torch.float32, device=dev)
+    ksum = torch.zeros((B, sp.kv_heads, D), dtype=torch.float32, device=dev)
+    qn, kn, kb, idx = sala.sparse_select(q, k, wq, wq, topk=sp.topk, n_init=sp.n_init,
+                                         n_local=sp.n_local)
+    k_cache[:, :N] = kn
+    v_cache[:, :N] = v
+    kbar[:, :N // 64] = kb
+    k_hist, v_hist = f64(k), f64(v)
+    ld = sala.linear_desc(B, 64, H, D)
+    sd = sala.sparse_desc(B, 64, sp.q_heads, sp.kv_heads, D, topk=sp.topk, n_init=sp.n_init,
+                          n_local=sp.n_local)
+    dd = sala.DecodeDesc(ld, sd, w.n_linear, cap)
+    ws = sala.workspace(sala.sala_decode_workspace_size(dd), dev)
+    worst = 0.0
+    for s in range(steps):
+        pos = N + s
+        tok = wl.decode_inputs(w, s, dev)
+        outs = [torch.empty_like(t[0]) for t in tok]
+        io = sala.make_decode_io(tok, outs, states, [lam] * w.n_linear, wq, wq)
+        st = sala.sala_decode_step(dd, io, k_cache, v_cache, kbar, ksum, pos, ws)
+        assert st == 0, sala.status_string(st)
+        torch.cuda.synchronize()
+        for l in range(w.n_linear):
+            tq, tk, tv, tg = (f64(t) for t in tok[l])
+            ro, ref_states[l] = oracle.decode_linear_step(ref_states[l], tq, tk, tv, tg, f64(lam),
+                                                          f64(wq), f64(wq), pos)
+            worst = max(worst, rel_err(f64(outs[l]), ro))
+        tq, tk, tv, tg = (f64(t) for t in tok[w.n_linear])
+        k_hist = np.concatenate([k_hist, tk[:, None]], axis=1)
+        v_hist = np.concatenate([v_hist, tv[:, None]], axis=1)
+        ro, _ = oracle.decode_sparse_step(k_hist, v_hist, tq, tg, f64(wq), f64(wq), pos,
+                                          topk=sp.topk, n_init=sp.n_init, n_local=sp.n_local)
+        worst = max(worst, rel_err(f64(outs[w.n_linear]), ro))
+    assert worst <= TOL, worst
+    for l in range(w.n_linear):
+        assert rel_err(f64(states[l]), ref_states[l]) <= TOL
+    assert sala.sala_get_device_status() == 0
