@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""SALA layer-group prefill benchmark on B200 (libsala).
+
+One step = one pass of the whole prefill hot path over one batch of
+synthetic input: three linear layers (sala_linear_prefill) and one sparse
+layer (sala_sparse_select + sala_sparse_prefill), inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload group_256k]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+single-GPU workload (the path is single-GPU; no collective on the data
+path); value = total tokens over all ranks / max-over-ranks time.  Prints
+one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from hybrid_sparse_linear_lightning_b200 import workloads as wl  # noqa: E402
+
+METRIC = "SALA layer-group prefill tokens/s at 256K on 1 B200; % bf16 tensor peak"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+def sparse_attn_flops(w: wl.Workload, N: int) -> float:
+    """4 * d * Hq FLOPs per visible (query, key) pair (QK^T and PV), summed over
+    the selected blocks of every query block: a full block gives 64*64 pairs,
+    the diagonal block 64*65/2."""
+    sp = w.sparse
+    nb = N // sp.block
+    pairs = 0
+    for i in range(nb):
+        # blocks attended by query block i: initial + local (overlapping near the
+        # start) + min(topk, candidates in [n_init, i - n_local])
+        first = min(sp.n_init, i + 1)
+        local = max(0, i - max(sp.n_init, i - sp.n_local + 1) + 1)
+        n = first + local + min(sp.topk, max(0, i - sp.n_local + 1 - sp.n_init))
+        pairs += (n - 1) * sp.block * sp.block + sp.block * (sp.block + 1) // 2
+    return float(pairs) * 4 * sp.head_dim * sp.q_heads * w.batch
+
+
+def linear_bytes(w: wl.Workload, N: int) -> float:
+    """Compulsory HBM bytes of one linear layer: Q, K, V, G read, O written."""
+    e = 2 if w.dtype == "bf16" else 4
+    return 5.0 * w.batch * N * w.linear.heads * w.linear.head_dim * e
+
+
+def select_bytes(w: wl.Workload, N: int) -> float:
+    """Q, K read; Q_norm, K_norm (bf16) written; block tables negligible."""
+    sp = w.sparse
+    e = 2 if w.dtype == "bf16" else 4
+    rows = w.batch * N * (sp.q_heads + sp.kv_heads) * sp.head_dim
+    return float(rows * (e + 2))
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        sm, mx, reasons = [], [], set()
+        for line in self.tmp.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.tmp.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class GroupPrefill:
+    """Pre-allocated inputs, outputs and workspaces of one layer group."""
+
+    def __init__(self, w: wl.Workload, N: int, dev, sala):
+        self.w, self.N, self.dev, self.sala = w, N, dev, sala
+        ln, sp = w.linear, w.sparse
+        B = w.batch
+        self.lin_inputs = [wl.layer_inputs(w, l, dev, seqlen=N) for l in range(w.n_linear)]
+        self.sp_inputs = wl.layer_inputs(w, w.n_linear, dev, seqlen=N)
+        self.lam = torch.tensor(wl.lam_schedule(ln), dtype=torch.float32, device=dev)
+        self.wt = wl.rms_weights(ln.head_dim, dev)
+        self.lin_out = [torch.empty_like(x[0]) for x in self.lin_inputs]
+        self.ld = sala.linear_desc(B, N, ln.heads, ln.head_dim, ln.chunk, w.torch_dtype)
+        self.sd = sala.sparse_desc(B, N, sp.q_heads, sp.kv_heads, sp.head_dim, sp.block, sp.topk,
+                                   sp.n_init, sp.n_local, w.torch_dtype)
+        self.lws = sala.workspace(sala.sala_linear_workspace_size(self.ld), dev)
+        self.sws = sala.workspace(sala.sala_sparse_workspace_size(self.sd), dev)
+        nb = N // sp.block
+        self.qn = torch.empty((B, N, sp.q_heads, sp.head_dim), dtype=torch.bfloat16, device=dev)
+        self.kn = torch.empty((B, N, sp.kv_heads, sp.head_dim), dtype=torch.bfloat16, device=dev)
+        self.kbar = torch.empty((B, nb, sp.kv_heads, sp.head_dim), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((B, sp.kv_heads, nb, sala.sala_sparse_index_width(self.sd)),
+                               dtype=torch.int32, device=dev)
+        self.sp_out = torch.empty_like(self.sp_inputs[0])
+        self.timers = None
+
+    def calls(self):
+        s = self.sala
+        res = []
+        for l in range(self.w.n_linear):
+            q, k, v, g = self.lin_inputs[l]
+            res.append(("linear_prefill", lambda q=q, k=k, v=v, g=g, l=l: s.sala_linear_prefill(
+                self.ld, q, k, v, g, self.lam, self.wt, self.wt, None, None, self.lin_out[l],
+                self.lws)))
+        q, k, v, g = self.sp_inputs
+        res.append(("sparse_select", lambda: s.sala_sparse_select(
+            self.sd, q, k, self.wt, self.wt, self.qn, self.kn, self.kbar, self.idx, self.sws)))
+        res.append(("sparse_prefill", lambda: s.sala_sparse_prefill(
+            self.sd, self.qn, self.kn, v, g, self.idx, self.sp_out)))
+        return res
+
+    def step(self, timed_calls=None):
+        for name, fn in self.calls():
+            if timed_calls is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            st = fn()
+            if st != 0:
+                raise RuntimeError(f"{name}: {self.sala.status_string(st)}")
+            if timed_calls is not None:
+                e1.record()
+                timed_calls.append((name, e0, e1))
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws <= 1:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, ws, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline_sample(w: wl.Workload, budget_s: float = 20.0):
+    """Time the oracle as it stands on a bounded sample of the workload.
+
+    Linear part: one linear layer, all heads, over the first T tokens (work per
+    token is constant).  Sparse part: the last q query blocks of a sequence of
+    Ns tokens (their selection is full).  Returns tokens/s of a layer group
+    extrapolated by work, the thread count and a description.
+    """
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = len(os.sched_getaffinity(0))
+    ln, sp = w.linear, w.sparse
+    f64 = lambda t: t.to(torch.float64).numpy()
+    T = 512 if budget_s < 15 else 1024
+    q, k, v, g = (f64(x) for x in wl.layer_inputs(w, 0, "cpu", seqlen=T))
+    lam = np.asarray(wl.lam_schedule(ln))
+    wt = np.ones(ln.head_dim)
+    t0 = time.perf_counter()
+    oracle.linear_layer(q, k, v, g, lam, wt, wt, chunk=ln.chunk)
+    t_lin = (time.perf_counter() - t0) / T
+    need = (sp.topk + sp.n_init + sp.n_local) * sp.block
+    Ns = max(4096, 2 * need)
+    nq = 2 if budget_s < 15 else 4
+    nb = Ns // sp.block
+    q, k, v, g = (f64(x) for x in wl.layer_inputs(w, w.n_linear, "cpu", seqlen=Ns))
+    t0 = time.perf_counter()
+    oracle.sparse_layer(q, k, v, g, wt, wt, block=sp.block, topk=sp.topk, n_init=sp.n_init,
+                        n_local=sp.n_local, query_blocks=list(range(nb - nq, nb)))
+    t_sp = (time.perf_counter() - t0) / (nq * sp.block)
+    per_token = w.n_linear * t_lin + t_sp
+    desc = (f"oracle (numpy fp64) on host cores: linear layer x{w.n_linear} timed on 1 layer x "
+            f"{ln.heads} heads x {T} tokens; sparse layer timed on the last {nq} query blocks "
+            f"of a {Ns}-token sequence (full top-{sp.topk} selection, scoring the whole prefix); "
+            f"tokens/s of the group extrapolated by per-token work")
+    return 1.0 / per_token, threads, desc, t_lin * T + t_sp * nq * sp.block
+
+
+def run_ours(args):
+    rank, ws, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from hybrid_sparse_linear_lightning_b200 import sala
+    w = wl.WORKLOADS[args.workload]
+    N = args.seqlen or w.seqlen
+    peaks, peak_kind = load_peaks()
+    grp = GroupPrefill(w, N, dev, sala)
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        grp.step()
+    torch.cuda.synchronize()
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(ws)
+    torch.cuda.synchronize()
+    launches0 = sala.sala_kernel_launch_count()
+    timed = []
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        grp.step(timed)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    launches = sala.sala_kernel_launch_count() - launches0
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), ws)
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    per_call = {}
+    for name, e0, e1 in timed:
+        per_call.setdefault(name, []).append(e0.elapsed_time(e1))
+    ms_per_step = elapsed_ms / args.steps
+    tokens = w.batch * N * ws * args.steps
+    value = tokens / (elapsed_ms / 1e3)
+
+    # per-call roofline (dominant call reported as "roofline")
+    calls = {}
+    work = {
+        "linear_prefill": ("hbm", linear_bytes(w, N)),
+        "sparse_select": ("hbm", select_bytes(w, N)),
+        "sparse_prefill": ("tensor", sparse_attn_flops(w, N)),
+    }
+    for name, ts in per_call.items():
+        avg = sum(ts) / len(ts)
+        bound, amount = work[name]
+        if bound == "hbm":
+            ach, pk, unit = amount / (avg / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            ach, pk, unit = amount / (avg / 1e3) / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
+        calls[name] = {"ms": round(avg, 4), "launches_per_step": ts and len(ts) // args.steps,
+                       "bound": bound, "achieved": round(ach, 2), "peak": pk, "unit": unit,
+                       "frac": round(ach / pk, 4), "share": 0.0}
+    tot = sum(c["ms"] * c["launches_per_step"] for c in calls.values())
+    for c in calls.values():
+        c["share"] = round(c["ms"] * c["launches_per_step"] / tot, 4)
+    dom = max(calls, key=lambda n: calls[n]["share"])
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            tr = json.load(f)
+        ent = tr.get(args.workload, {}).get(dom)
+        if ent and ent.get("kernel_version") == sala.sala_version():
+            traffic = ent["bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
+    d = calls[dom]
+    roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
+                "unit": d["unit"], "frac": d["frac"], "traffic": traffic, "kernel": dom,
+                "peak_source": f"{peak_kind} ({'sustained bf16' if d['bound'] == 'tensor' else 'HBM copy'})"}
+
+    # end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(grp, args, ws)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, threads, desc, secs = cpu_baseline_sample(w, args.cpu_budget)
+        cpu = {"value": round(v, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc, "sample_seconds": round(secs, 2)}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic N(0,1) inputs, seeded (no trained weights)",
+            "config": {"workload": w.name, "seq_len": N, "batch": w.batch,
+                       "layers": f"{w.n_linear} linear + 1 sparse",
+                       "heads": w.linear.heads, "kv_heads": w.sparse.kv_heads,
+                       "head_dim": w.linear.head_dim, "chunk": w.linear.chunk,
+                       "block": w.sparse.block, "topk": w.sparse.topk,
+                       "n_init": w.sparse.n_init, "n_local": w.sparse.n_local,
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (no flush needed)"},
+            "roofline": roofline, "calls": calls,
+            "tensor_frac_of_step": round(sparse_attn_flops(w, N) / (ms_per_step / 1e3) / 1e12
+                                         / peaks["bf16_tflops_sustained"], 4),
+            "e2e": e2e, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
+        }
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(grp: GroupPrefill, args, ws):
+    """Same step through the C ABI, inputs copied from pinned host memory and
+    outputs read back inside the timed region."""
+    w, N = grp.w, grp.N
+    host_in = []
+    for tens in grp.lin_inputs + [grp.sp_inputs]:
+        host_in.append([t.to("cpu").pin_memory() for t in tens])
+    host_out = [o.to("cpu").pin_memory() for o in grp.lin_out + [grp.sp_out]]
+    dev_in = grp.lin_inputs + [grp.sp_inputs]
+    dev_out = grp.lin_out + [grp.sp_out]
+    h2d = sum(t.numel() * t.element_size() for ts in host_in for t in ts)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def one():
+        for hs, ds in zip(host_in, dev_in):
+            for h, d in zip(hs, ds):
+                d.copy_(h, non_blocking=True)
+        grp.step()
+        for d, h in zip(dev_out, host_out):
+            h.copy_(d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(ws)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e), ws)
+    barrier(ws)
+    return {"value": round(w.batch * N * ws * steps / (ms / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        cpu_baseline_sample(w, budget_s=5.0)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        v, threads, desc, s = cpu_baseline_sample(w, budget_s=5.0)
+        vals.append(v)
+        secs += s
+    value = len(vals) / sum(1.0 / v for v in vals)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 / value, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic N(0,1) inputs, seeded (no trained weights)",
+        "config": {"workload": w.name, "seq_len": w.seqlen, "batch": w.batch,
+                   "layers": f"{w.n_linear} linear + 1 sparse"},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="group_256k", choices=list(wl.WORKLOADS))
+    ap.add_argument("--seqlen", type=int, default=0, help="override the workload length")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

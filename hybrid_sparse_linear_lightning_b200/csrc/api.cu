@@ -5,6 +5,7 @@
 // synchronously; launches go to the caller's stream.  The library allocates
 // no memory: scratch lives in the caller's workspace.
 #include <algorithm>
+#include <atomic>
 #include <math.h>
 #include <string.h>
 
@@ -28,7 +29,11 @@ inline bool aligned16_or_null(const void* p) { return !p || ((uintptr_t)p & 15u)
 
 inline size_t elt_size(sala_dtype t) { return t == SALA_F32 ? 4 : 2; }
 
+std::atomic<uint64_t> g_launches{0};
+
+// Called once after every kernel launch: counts it and maps the launch error.
 inline sala_status launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? SALA_OK : SALA_ERR_CUDA;
 }
 
@@ -372,5 +377,7 @@ sala_status sala_get_device_status(void* stream) {
 }
 
 int sala_version(void) { return 100; }
+
+uint64_t sala_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

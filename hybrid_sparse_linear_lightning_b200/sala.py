@@ -32,7 +32,7 @@ EXPORTED = [
     "sala_sparse_index_width", "sala_linear_workspace_size", "sala_linear_prefill",
     "sala_sparse_workspace_size", "sala_sparse_select", "sala_sparse_prefill",
     "sala_decode_workspace_size", "sala_decode_step", "sala_status_string",
-    "sala_get_device_status", "sala_version",
+    "sala_get_device_status", "sala_version", "sala_kernel_launch_count",
 ]
 
 
@@ -89,6 +89,7 @@ def _load():
         "sala_status_string": (ctypes.c_char_p, [I]),
         "sala_get_device_status": (I, [P]),
         "sala_version": (I, []),
+        "sala_kernel_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -200,6 +201,10 @@ def sala_get_device_status(stream=None) -> int:
 
 def sala_version() -> int:
     return int(LIB.sala_version())
+
+
+def sala_kernel_launch_count() -> int:
+    return int(LIB.sala_kernel_launch_count())
 
 
 # ---------------------------------------------------------------------------- tensor helpers

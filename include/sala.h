@@ -183,6 +183,10 @@ sala_status sala_get_device_status(void* stream);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int sala_version(void);
 
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all entry points), for launch accounting by callers. */
+uint64_t sala_kernel_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
