@@ -6,6 +6,7 @@
 // no memory: scratch lives in the caller's workspace.
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <math.h>
 #include <string.h>
 
@@ -26,8 +27,6 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 inline bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
 inline bool aligned16_or_null(const void* p) { return !p || ((uintptr_t)p & 15u) == 0; }
-
-inline size_t elt_size(sala_dtype t) { return t == SALA_F32 ? 4 : 2; }
 
 std::atomic<uint64_t> g_launches{0};
 
@@ -233,6 +232,40 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free selection (sala_sparse_select_noalloc).
+//
+// Some callers cannot call cudaMalloc at all: code running inside an
+// allocator-free runtime or a memory pool that forbids extra device
+// allocations, or a host that must not allocate while a stream is being
+// captured.  For them the selection's scratch (the group-summed query block
+// means, B * (N/block) * Hkv * head_dim fp32 values) lives in this
+// file-scope device array instead of a caller workspace.  It is loaded with
+// the library and stays resident on every GPU that loads it until the
+// process exits.
+constexpr size_t kNoAllocScratchBytes = SALA_NOALLOC_SCRATCH_BYTES;   // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  Host code only
+// sees a host-side stand-in under that name, so the address is looked up
+// once per device (with that device current) and cached.
+sala_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SALA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SALA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SALA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -317,6 +350,32 @@ sala_status sala_sparse_prefill(const sala_sparse_desc* d, const void* q_norm,
   if (d->head_dim == 128)
     return run_sparse_prefill<float, 128>(d, q_norm, k_norm, v, gate, idx, out, st);
   return run_sparse_prefill<float, 64>(d, q_norm, k_norm, v, gate, idx, out, st);
+}
+
+sala_status sala_sparse_select_noalloc(const sala_sparse_desc* d, const void* q, const void* k,
+                                       const float* wq, const float* wk, void* q_norm,
+                                       void* k_norm, float* kbar, int32_t* idx, void* stream) {
+  sala_status s = check_sparse(d);
+  if (s != SALA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(wq) || !aligned16(wk) || !aligned16(q_norm) ||
+      !aligned16(k_norm) || !aligned16(kbar) || !aligned16(idx))
+    return SALA_ERR_INVALID_ARG;
+  // The scratch is written in full by the normalisation kernel before the
+  // scoring kernel reads it, so nothing in it has to start at zero.
+  if (sala_sparse_workspace_size(d) > kNoAllocScratchBytes) return SALA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != SALA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(scratch);
+  if (d->dtype == SALA_BF16) {
+    if (d->head_dim == 128)
+      return run_select<__nv_bfloat16, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+    return run_select<__nv_bfloat16, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+  }
+  if (d->head_dim == 128)
+    return run_select<float, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+  return run_select<float, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
 }
 
 size_t sala_decode_workspace_size(const sala_decode_desc* d) {

@@ -33,7 +33,9 @@ EXPORTED = [
     "sala_sparse_workspace_size", "sala_sparse_select", "sala_sparse_prefill",
     "sala_decode_workspace_size", "sala_decode_step", "sala_status_string",
     "sala_get_device_status", "sala_version", "sala_kernel_launch_count",
+    "sala_sparse_select_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class SalaError(RuntimeError):
@@ -90,6 +92,7 @@ def _load():
         "sala_get_device_status": (I, [P]),
         "sala_version": (I, []),
         "sala_kernel_launch_count": (ctypes.c_uint64, []),
+        "sala_sparse_select_noalloc": (I, [P] + [P] * 8 + [P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -173,6 +176,17 @@ def sala_sparse_select(d: SparseDesc, q, k, wq, wk, q_norm, k_norm, kbar, idx, w
     return LIB.sala_sparse_select(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
                                   _ptr(q_norm), _ptr(k_norm), _ptr(kbar), _ptr(idx),
                                   _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def sala_sparse_select_noalloc(d: SparseDesc, q, k, wq, wk, q_norm, k_norm, kbar, idx,
+                               stream=None) -> int:
+    """sala_sparse_select without a workspace: for callers that cannot allocate
+    device memory.  Its scratch is a fixed 4 MiB array inside the library
+    (shapes needing more return SALA_ERR_WORKSPACE); calls on one device must
+    not overlap on the GPU."""
+    return LIB.sala_sparse_select_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
+                                          _ptr(q_norm), _ptr(k_norm), _ptr(kbar), _ptr(idx),
+                                          _stream(stream))
 
 
 def sala_sparse_prefill(d: SparseDesc, q_norm, k_norm, v, gate, idx, out, workspace=None,

@@ -117,6 +117,30 @@ sala_status sala_sparse_select(const sala_sparse_desc* d, const void* q, const v
                                float* kbar, int32_t* idx, void* workspace, size_t ws_bytes,
                                void* stream);
 
+/* Allocation-free variant of sala_sparse_select (no counterpart on the
+ * pages: it exists for callers, not for the method).  Same arguments and
+ * results, minus the workspace: its scratch is a fixed array of
+ * SALA_NOALLOC_SCRATCH_BYTES (4 MiB) compiled into the library, which every
+ * GPU that loads the library keeps until the process exits.  It serves
+ * callers that cannot allocate device memory, e.g. code inside an
+ * allocator-free runtime or a memory pool that forbids new allocations.
+ *   - Limit: sala_sparse_workspace_size(d) must not exceed the array size
+ *     (batch * seqlen/block * kv_heads * head_dim * 4 bytes; 262144 tokens
+ *     at batch 1, 2 kv heads, head_dim 128); larger shapes return
+ *     SALA_ERR_WORKSPACE and launch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture on the device.
+ *   - The library calls no cudaMalloc / cudaFree here.
+ *   - All calls on one device share the array, so calls that may overlap on
+ *     the GPU (different streams without ordering) race and must not be
+ *     issued; calls ordered on one stream are safe.  The array keeps the
+ *     last call's contents; each call overwrites what it reads. */
+#define SALA_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+sala_status sala_sparse_select_noalloc(const sala_sparse_desc* d, const void* q, const void* k,
+                                       const float* wq, const float* wk, void* q_norm,
+                                       void* k_norm, float* kbar, int32_t* idx, void* stream);
+
 /* Gathered block-sparse attention with the sigmoid gate.
  * In:  q_norm [B, N, Hq, d] bf16, k_norm [B, N, Hkv, d] bf16 (as written by
  *      sala_sparse_select), v [B, N, Hkv, d] and gate [B, N, Hq, d] of
