@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 #include <math.h>
 #include <string.h>
 
@@ -17,6 +18,9 @@
 #include "prologue.cuh"
 #include "select.cuh"
 #include "sparse_simt.cuh"
+#include "sparse_tc.cuh"
+
+#include <cudaTypedefs.h>
 
 using namespace sala;
 
@@ -124,10 +128,67 @@ sala_status run_select(const sala_sparse_desc* d, const void* q, const void* k, 
   return launch_status();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 view [rows, cols] (cols contiguous) with 64 x 64 boxes, 128-byte
+// swizzle: one box fills a 64-row x 128-byte tile of an MMA operand.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+sala_status run_sparse_prefill_tc(const sala_sparse_desc* d, const void* qn, const void* kn,
+                                  const void* v, const void* gate, const int32_t* idx, void* out,
+                                  cudaStream_t st) {
+  const int nb = d->seqlen / d->block;
+  const uint64_t rows = (uint64_t)d->batch * d->seqlen;
+  CUtensorMap qm, km, vm;
+  if (!make_tmap_bf16(&qm, qn, (uint64_t)d->q_heads * D, rows) ||
+      !make_tmap_bf16(&km, kn, (uint64_t)d->kv_heads * D, rows) ||
+      !make_tmap_bf16(&vm, v, (uint64_t)d->kv_heads * D, rows))
+    return SALA_ERR_CUDA;
+  const int width = d->topk + d->n_init + d->n_local;
+  const size_t smem = SpTcLayout<D>::kBytes(width) + 1024;
+  auto kern = sparse_attn_tc_kernel<__nv_bfloat16, D>;
+  if (allow_smem(kern, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  const int G = d->q_heads / d->kv_heads;
+  const long long grid = (long long)d->batch * d->kv_heads * nb * (G / kSpTcHeadsPerCta);
+  const float sl2 = sparse_scale(d) * 1.4426950408889634f;
+  kern<<<(unsigned)grid, kSpTcThreads, smem, st>>>(
+      qm, km, vm, idx, static_cast<const __nv_bfloat16*>(gate), static_cast<__nv_bfloat16*>(out),
+      d->seqlen, d->q_heads, d->kv_heads, width, sl2);
+  return launch_status();
+}
+
 template <typename T, int D>
 sala_status run_sparse_prefill(const sala_sparse_desc* d, const void* qn, const void* kn,
                                const void* v, const void* gate, const int32_t* idx, void* out,
                                cudaStream_t st) {
+  // bf16 activations with a GQA group of a multiple of 4 q heads run on the
+  // tensor cores; other shapes (fp32 activations, small groups) on CUDA cores.
+  if (std::is_same<T, __nv_bfloat16>::value && (d->q_heads / d->kv_heads) % kSpTcHeadsPerCta == 0)
+    return run_sparse_prefill_tc<D>(d, qn, kn, v, gate, idx, out, st);
   const int nb = d->seqlen / d->block;
   const size_t smem = sizeof(SpSimtSmem<D>);
   if (allow_smem(sparse_attn_simt_kernel<T, D>, smem) != cudaSuccess) return SALA_ERR_CUDA;

@@ -1,0 +1,307 @@
+// Gathered block-sparse attention on the 5th-generation tensor cores.
+//
+// InfLLM-V2-style sparse layer (acgfav.com "SALA 混合架构": each query
+// attends to a small set of selected key blocks), NoPE, output gate after the
+// block (MiniCPM-SALA paper, summary).  For query block i of kv head g, the
+// 64 tokens of every q head of the group share one list of selected key
+// blocks, so a CTA takes FOUR q heads of the group (two 128-row tiles: 2 heads
+// x 64 tokens each) and streams each selected K/V block through shared memory
+// once for all 256 query rows (GQA sharing without multicast).
+//
+// Per selected block j (64 keys):  S_t = Q_t K_j^T  (tcgen05, M=128 N=64,
+// fp32 in TMEM);  softmax warps read S_t one row per thread, apply the causal
+// mask on the diagonal block, exponentiate against a running max, write
+// P_t (bf16) to shared memory;  O_t += P_t V_j  (tcgen05, M=128 N=d, fp32 in
+// TMEM).  Exact softmax: the running max is raised (and O, l rescaled) only
+// when a row's max grows by more than 2^8, so values stay bounded; the final
+// division by l makes the result independent of that choice up to rounding.
+// Epilogue: out = sigmoid(gate) * O / l.
+//
+// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 issues MMAs (one
+// elected thread), warp 2 owns the TMEM allocation, warps 4-7 / 8-11 are the
+// softmax + epilogue warpgroups of tile 0 / tile 1.  Every mbarrier wait is
+// bounded; a wait that runs out sets the device status word and the CTA
+// winds down without touching further data.
+#pragma once
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace sala {
+
+constexpr int kSpTcThreads = 384;
+constexpr int kSpTcStages = 3;
+constexpr int kSpTcHeadsPerCta = 4;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+template <int D>
+struct SpTcLayout {
+  static constexpr int kAtoms = D / 64;                 // 128-byte column atoms of a row
+  static constexpr int kQTile = 128 * D * 2;            // one 128-row Q tile
+  static constexpr int kKV = 64 * D * 2;                // one 64-row K or V block
+  static constexpr int kP = 128 * 64 * 2;               // one P tile
+  static constexpr int kQ = 0;
+  static constexpr int kKVBase = kQ + 2 * kQTile;
+  static constexpr int kPBase = kKVBase + kSpTcStages * 2 * kKV;
+  static constexpr int kBar = kPBase + 2 * kP;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_done[2], fin
+  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 8 + 1;
+  static constexpr int kMisc = kBar + 8 * kNumBars;
+  static constexpr int kSel = kMisc + 16;               // int sel[width]
+  static constexpr int kBytes(int width) { return kSel + 4 * width; }
+  static constexpr int kTmemCols = D == 128 ? 512 : 256;
+  // TMEM columns: S_0, S_1 (64 each), O_0, O_1 (D each)
+  static constexpr int kColS0 = 0, kColS1 = 64, kColO0 = 128, kColO1 = 128 + D;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSpTcThreads, 1)
+sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                      const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap,
+                      const int32_t* __restrict__ idx, const T* __restrict__ gate,
+                      T* __restrict__ out, int N, int Hq, int Hkv, int width, float sl2) {
+  using L = SpTcLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + kSpTcStages;
+  uint64_t* s_full = kv_empty + kSpTcStages;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* fin = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  int* n_sel_slot = reinterpret_cast<int*>(smem + L::kMisc + 4);
+  int* sel = reinterpret_cast<int*>(smem + L::kSel);
+
+  const int G = Hq / Hkv;
+  const int nq = G / kSpTcHeadsPerCta;
+  const int nb = N / 64;
+  const int hq = blockIdx.x % nq;
+  const int i = (blockIdx.x / nq) % nb;
+  const int g = (blockIdx.x / (nq * nb)) % Hkv;
+  const int b = blockIdx.x / (nq * nb * Hkv);
+  const int hbase = g * G + hq * kSpTcHeadsPerCta;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- setup: barriers, TMEM, the block list
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int s = 0; s < kSpTcStages; ++s) {
+      tc::mbar_init(kv_full + s, 1);
+      tc::mbar_init(kv_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      tc::mbar_init(s_full + t, 1);
+      tc::mbar_init(s_free + t, 4);
+      tc::mbar_init(p_full + t, 4);
+      tc::mbar_init(o_done + t, 1);
+    }
+    tc::mbar_init(fin, 1);
+    tc::fence_barrier_init();
+    // valid prefix of the ascending index row (entries in [0, i])
+    const int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
+    int n = 0, prev = -1;
+    for (int e = 0; e < width; ++e) {
+      const int j = row[e];
+      if (j < 0) break;
+      if (j > i || j <= prev) { set_status(kStatusBounds); break; }
+      sel[n++] = j;
+      prev = j;
+    }
+    *n_sel_slot = n;
+  }
+  if (warp == 2) {
+    tc::tmem_alloc(tmem_slot, L::kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_sel = *n_sel_slot;
+
+  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sKV = smem + L::kKVBase;
+  uint8_t* sP = smem + L::kPBase;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (tc::elect_one() && n_sel > 0) {
+      tc::tma_prefetch(&qmap);
+      tc::tma_prefetch(&kmap);
+      tc::tma_prefetch(&vmap);
+      tc::mbar_expect_tx(q_full, 2 * L::kQTile);
+      const int row0 = b * N + i * 64;
+      for (int t = 0; t < 2; ++t)
+        for (int hl = 0; hl < 2; ++hl)
+          for (int a = 0; a < L::kAtoms; ++a)
+            tc::tma_load_2d(sQ + t * L::kQTile + a * (128 * 128) + hl * (64 * 128), &qmap, q_full,
+                            (hbase + 2 * t + hl) * D + 64 * a, row0);
+      for (int j = 0; j < n_sel; ++j) {
+        const int st = j % kSpTcStages, use = j / kSpTcStages;
+        if (use > 0 && !tc::mbar_wait(kv_empty + st, (use - 1) & 1)) break;
+        tc::mbar_expect_tx(kv_full + st, 2 * L::kKV);
+        uint8_t* k_dst = sKV + st * 2 * L::kKV;
+        uint8_t* v_dst = k_dst + L::kKV;
+        const int krow = b * N + sel[j] * 64;
+        for (int a = 0; a < L::kAtoms; ++a) {
+          tc::tma_load_2d(k_dst + a * (64 * 128), &kmap, kv_full + st, g * D + 64 * a, krow);
+          tc::tma_load_2d(v_dst + a * (64 * 128), &vmap, kv_full + st, g * D + 64 * a, krow);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (tc::elect_one() && n_sel > 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = tc::smem_u32(sQ), kv_addr = tc::smem_u32(sKV),
+                     p_addr = tc::smem_u32(sP);
+      bool ok = tc::mbar_wait(q_full, 0);
+      for (int j = 0; ok && j < n_sel; ++j) {
+        const int st = j % kSpTcStages;
+        if (!(ok = tc::mbar_wait(kv_full + st, (j / kSpTcStages) & 1))) break;
+        tc::tc_fence_after();
+        const uint32_t k_addr = kv_addr + st * 2 * L::kKV, v_addr = k_addr + L::kKV;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j > 0 && !(ok = tc::mbar_wait(s_free + t, (j - 1) & 1))) break;
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;   // 16 elements = 32 B inside the atom
+            const uint64_t ad = tc::smem_desc_sw128(q_addr + t * L::kQTile + (kk >> 2) * (128 * 128) + off, 16, 1024);
+            const uint64_t bd = tc::smem_desc_sw128(k_addr + (kk >> 2) * (64 * 128) + off, 16, 1024);
+            tc::mma_bf16_ss(tmem + (t ? L::kColS1 : L::kColS0), ad, bd, idesc_s, kk > 0);
+          }
+          tc::mma_commit(s_full + t);
+        }
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = tc::mbar_wait(p_full + t, j & 1))) break;
+          tc::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = tc::smem_desc_sw128(p_addr + t * L::kP + kk * 32, 16, 1024);
+            const uint64_t bd = tc::smem_desc_sw128(v_addr + kk * 2048, 64 * 128, 1024);
+            tc::mma_bf16_ss(tmem + (t ? L::kColO1 : L::kColO0), ad, bd, idesc_o, (j > 0 || kk > 0));
+          }
+          tc::mma_commit(o_done + t);
+        }
+        if (ok) tc::mma_commit(kv_empty + st);
+      }
+      // drain: every MMA issued above has completed once `fin` fires
+      tc::mma_commit(fin);
+      tc::mbar_wait(fin, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = (warp - 4) >> 2;            // tile
+    const int quad = warp & 3;                // TMEM lane quadrant
+    const int r = quad * 32 + lane;           // row in the tile
+    const int tok = r & 63;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t s_addr = lane_base + (t ? L::kColS1 : L::kColS0);
+    const uint32_t o_addr = lane_base + (t ? L::kColO1 : L::kColO0);
+    uint8_t* p_row = sP + t * L::kP + r * 128;
+    float m = -INFINITY, l = 0.f;
+    bool ok = n_sel > 0;
+    for (int j = 0; ok && j < n_sel; ++j) {
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(s_full + t, j & 1));
+      if (!ok) break;
+      tc::tc_fence_after();
+      float x[64];
+      tc::tmem_ld32(s_addr, x);
+      tc::tmem_ld32(s_addr + 32, x + 32);
+      tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(s_free + t);
+      const bool diag = sel[j] == i;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = (diag && c > tok) ? -INFINITY : x[c] * sl2;
+        mx = fmaxf(mx, x[c]);
+      }
+      if (j == 0) m = mx;
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
+        if (!ok) break;
+        if (__any_sync(0xffffffffu, mx > m + kRescaleThreshold)) {
+          const float mnew = fmaxf(m, mx);
+          const float f = exp2f(m - mnew);
+          m = mnew;
+          l *= f;
+          tc::tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float o[32];
+            tc::tmem_ld32(o_addr + c0, o);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= f;
+            tc::tmem_st32(o_addr + c0, o);
+          }
+          tc::tmem_wait_st();
+        }
+      }
+      // P = exp2(x - m) as bf16, written in the 128B-swizzled K-major layout
+      float rs = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        float pv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pv[e] = exp2f(x[ch * 8 + e] - m);
+          rs += pv[e];
+        }
+        uint4 u;
+        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
+        *reinterpret_cast<uint4*>(p_row + ((ch ^ (r & 7)) << 4)) = u;
+      }
+      l += rs;
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(p_full + t);
+    }
+    // epilogue: out = sigmoid(gate) * O / l
+    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (n_sel - 1) & 1));
+    if (ok) {
+      tc::tc_fence_after();
+      const int head = hbase + 2 * t + (r >> 6);
+      const long long off = (((long long)b * N + (long long)i * 64 + tok) * Hq + head) * D;
+      const float inv_l = 1.f / l;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float o[32];
+        tc::tmem_ld32(o_addr + c0, o);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          float gv[8];
+          load8(gate + off + c0 + c, gv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) gv[e] = sigmoidf_(gv[e]) * o[c + e] * inv_l;
+          store8(out + off + c0 + c, gv);
+        }
+      }
+    }
+  }
+
+  // ---- teardown
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace sala

@@ -143,6 +143,13 @@ def test_sparse_tiny_f32(sala):
     assert _compare_sparse(r, w.sparse) == 0
 
 
+def test_sparse_tiny_bf16_d64(sala):
+    w = _w("tiny_2k_f32", dtype="bf16")
+    r = run_sparse_case(sala, w)
+    assert r["out"].dtype == torch.bfloat16
+    _compare_sparse(r, w.sparse)
+
+
 @pytest.mark.parametrize("seqlen,topk,n_local", [(4160, 16, 2), (8192, 64, 4)])
 def test_sparse_bf16_d128(sala, seqlen, topk, n_local):
     w = _w("group_32k", sparse={"topk": topk, "n_local": n_local})
