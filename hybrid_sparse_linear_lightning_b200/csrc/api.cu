@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "linear_simt.cuh"
+#include "linear_tc.cuh"
 #include "prologue.cuh"
 #include "select.cuh"
 #include "sparse_simt.cuh"
@@ -86,6 +87,11 @@ LinearWs linear_ws(const sala_linear_desc* d) {
   return w;
 }
 
+sala_status run_linear_tc(const sala_linear_desc* d, const __nv_bfloat16* qn,
+                          const __nv_bfloat16* kn, const void* v, const void* gate,
+                          const float* lambda, const float* state_in, float* state_out, void* out,
+                          cudaStream_t st);
+
 template <typename T, int D>
 sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, const void* v,
                        const void* gate, const float* lambda, const float* wq, const float* wk,
@@ -100,6 +106,10 @@ sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, 
       static_cast<const T*>(q), static_cast<const T*>(k), wq, wk, qn, kn, tokens, d->seqlen,
       d->heads, d->pos0, log2((double)d->rope_base), d->rms_eps);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  // bf16 activations with head_dim 128 run on the tensor cores; fp32
+  // activations and head_dim 64 on CUDA cores.
+  if (std::is_same<T, __nv_bfloat16>::value && D == 128)
+    return run_linear_tc(d, qn, kn, v, gate, lambda, state_in, state_out, out, st);
   const size_t smem = sizeof(SimtSmem<D>);
   if (allow_smem(linear_chunk_simt_kernel<T, D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
   const int grid = d->batch * d->heads * (D / kSimtCols);
@@ -143,18 +153,44 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// 2D bf16 view [rows, cols] (cols contiguous) with 64 x 64 boxes, 128-byte
-// swizzle: one box fills a 64-row x 128-byte tile of an MMA operand.
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows) {
+// 2D bf16 view [rows, cols] (cols contiguous) loaded in boxes of
+// box_cols x box_rows.  With 128-byte swizzle and 64-column boxes one box
+// fills box_rows x 128 B of a K-major or MN-major MMA operand; with 64-byte
+// swizzle and 32-column boxes, box_rows x 64 B.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                    uint32_t box_cols = 64, uint32_t box_rows = 64,
+                    CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+sala_status run_linear_tc(const sala_linear_desc* d, const __nv_bfloat16* qn,
+                          const __nv_bfloat16* kn, const void* v, const void* gate,
+                          const float* lambda, const float* state_in, float* state_out, void* out,
+                          cudaStream_t st) {
+  constexpr int D = 128;
+  const uint64_t rows = (uint64_t)d->batch * d->seqlen, cols = (uint64_t)d->heads * D;
+  CUtensorMap qm, km, vm;
+  if (!make_tmap_bf16(&qm, qn, cols, rows, 64, kLinTile) ||
+      !make_tmap_bf16(&km, kn, cols, rows, 64, kLinTile) ||
+      !make_tmap_bf16(&vm, v, cols, rows, kLinCols, kLinTile, CU_TENSOR_MAP_SWIZZLE_64B))
+    return SALA_ERR_CUDA;
+  const size_t smem = LinTcLayout::kBytes + 1024;
+  auto kern = linear_attn_tc_kernel<__nv_bfloat16>;
+  if (allow_smem(kern, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  const int grid = d->batch * d->heads * (D / kLinCols);
+  kern<<<grid, kLinTcThreads, smem, st>>>(qm, km, vm, static_cast<const __nv_bfloat16*>(gate),
+                                          lambda, state_in, state_out,
+                                          static_cast<__nv_bfloat16*>(out), d->seqlen, d->heads,
+                                          d->scale);
+  return launch_status();
 }
 
 template <int D>
