@@ -62,8 +62,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                       const int32_t* __restrict__ idx, const T* __restrict__ gate,
                       T* __restrict__ out, int N, int Hq, int Hkv, int width, float sl2) {
   using L = SpTcLayout<D>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+  extern __shared__ __align__(1024) uint8_t smem_tc[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_tc) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* q_full = bars;
@@ -162,36 +162,49 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = tc::smem_u32(sQ), kv_addr = tc::smem_u32(sKV),
                      p_addr = tc::smem_u32(sP);
-      bool ok = tc::mbar_wait(q_full, 0);
-      for (int j = 0; ok && j < n_sel; ++j) {
-        const int st = j % kSpTcStages;
-        if (!(ok = tc::mbar_wait(kv_full + st, (j / kSpTcStages) & 1))) break;
-        tc::tc_fence_after();
-        const uint32_t k_addr = kv_addr + st * 2 * L::kKV, v_addr = k_addr + L::kKV;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j > 0 && !(ok = tc::mbar_wait(s_free + t, (j - 1) & 1))) break;
-          tc::tc_fence_after();
+      // Issue order: S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...  so the
+      // softmax of one tile overlaps the tensor work of the other.
+      auto issue_s = [&](int t, int j) {
+        const uint32_t k_addr = kv_addr + (j % kSpTcStages) * 2 * L::kKV;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;   // 16 elements = 32 B inside the atom
-            const uint64_t ad = tc::smem_desc_sw128(q_addr + t * L::kQTile + (kk >> 2) * (128 * 128) + off, 16, 1024);
-            const uint64_t bd = tc::smem_desc_sw128(k_addr + (kk >> 2) * (64 * 128) + off, 16, 1024);
-            tc::mma_bf16_ss(tmem + (t ? L::kColS1 : L::kColS0), ad, bd, idesc_s, kk > 0);
-          }
-          tc::mma_commit(s_full + t);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;   // 16 elements = 32 B inside the atom
+          const uint64_t ad = tc::smem_desc_sw128(q_addr + t * L::kQTile + (kk >> 2) * (128 * 128) + off, 16, 1024);
+          const uint64_t bd = tc::smem_desc_sw128(k_addr + (kk >> 2) * (64 * 128) + off, 16, 1024);
+          tc::mma_bf16_ss(tmem + (t ? L::kColS1 : L::kColS0), ad, bd, idesc_s, kk > 0);
         }
+        tc::mma_commit(s_full + t);
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t v_addr = kv_addr + (j % kSpTcStages) * 2 * L::kKV + L::kKV;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = tc::smem_desc_sw128(p_addr + t * L::kP + kk * 32, 16, 1024);
+          const uint64_t bd = tc::smem_desc_sw128(v_addr + kk * 2048, 64 * 128, 1024);
+          tc::mma_bf16_ss(tmem + (t ? L::kColO1 : L::kColO0), ad, bd, idesc_o, (j > 0 || kk > 0));
+        }
+        tc::mma_commit(o_done + t);
+      };
+      bool ok = tc::mbar_wait(q_full, 0) && tc::mbar_wait(kv_full, 0);
+      if (ok) {
+        tc::tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int j = 0; ok && j < n_sel; ++j) {
+        const bool more = j + 1 < n_sel;
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = tc::mbar_wait(p_full + t, j & 1))) break;
           tc::tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = tc::smem_desc_sw128(p_addr + t * L::kP + kk * 32, 16, 1024);
-            const uint64_t bd = tc::smem_desc_sw128(v_addr + kk * 2048, 64 * 128, 1024);
-            tc::mma_bf16_ss(tmem + (t ? L::kColO1 : L::kColO0), ad, bd, idesc_o, (j > 0 || kk > 0));
+          issue_pv(t, j);
+          if (t == 1) tc::mma_commit(kv_empty + (j % kSpTcStages));
+          if (more) {
+            if (t == 0 && !(ok = tc::mbar_wait(kv_full + (j + 1) % kSpTcStages, ((j + 1) / kSpTcStages) & 1))) break;
+            if (!(ok = tc::mbar_wait(s_free + t, j & 1))) break;
+            tc::tc_fence_after();
+            issue_s(t, j + 1);
           }
-          tc::mma_commit(o_done + t);
         }
-        if (ok) tc::mma_commit(kv_empty + st);
       }
       // drain: every MMA issued above has completed once `fin` fires
       tc::mma_commit(fin);
@@ -220,13 +233,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_free + t);
-      const bool diag = sel[j] == i;
-      float mx = -INFINITY;
+      // causal mask on the diagonal block only (warp-uniform branch); the max
+      // is taken on raw logits and scaled once (sl2 > 0)
+      if (sel[j] == i) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        x[c] = (diag && c > tok) ? -INFINITY : x[c] * sl2;
-        mx = fmaxf(mx, x[c]);
+        for (int c = 0; c < 64; ++c) x[c] = c > tok ? -INFINITY : x[c];
       }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+      mx *= sl2;
       if (j == 0) m = mx;
       if (j > 0) {
         ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
@@ -256,7 +272,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         float pv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          pv[e] = exp2f(x[ch * 8 + e] - m);
+          pv[e] = exp2f(fmaf(x[ch * 8 + e], sl2, -m));
           rs += pv[e];
         }
         uint4 u;
