@@ -18,12 +18,13 @@
 // thread); a bf16 copy is written to shared memory as the B operand of the
 // next tile's Q^ S product.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one
-// elected thread), warps 4-7 build V' and the diagonal 32-column chunks of
-// P, warps 2-3 (also the TMEM owner) and warps 6-7 the off-diagonal chunks,
-// warps 8-11 update the state and run the gated epilogue.  The QK, dS and O
-// accumulators are double-buffered in TMEM so the tensor work of tile c+1
-// overlaps the element-wise work of tile c.  Waits are bounded.
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 MMA issuer (one
+// elected thread), warps 2-7 build P (balanced 32-column chunks; warp 2 also
+// owns TMEM) and write it to TMEM as the A operand of P V, warps 8-11 update
+// the state and build V' for the next tile (the short chain that feeds the
+// next dS and Q S products), warps 12-15 run the gated epilogue.  The QK, dS
+// and O accumulators are double-buffered in TMEM so the tensor work of tile
+// c+1 overlaps the element-wise work of tile c.  Waits are bounded.
 #pragma once
 
 #include "common.cuh"
@@ -31,25 +32,25 @@
 
 namespace sala {
 
-constexpr int kLinTcThreads = 384;
+constexpr int kLinTcThreads = 512;
 constexpr int kLinTile = 128;
 constexpr int kLinCols = 32;
 constexpr int kLinStages = 2;
 
 struct LinTcLayout {
-  // per stage: Q^ tile (2 atoms x 16 KB), K^ tile (same), V slice (128 rows x 64 B)
+  // per stage: Q^ tile and K^ tile (2 atoms x 16 KB each); V slices in their own ring
   static constexpr int kQ = 0;
   static constexpr int kK = 32768;
-  static constexpr int kV = 65536;
-  static constexpr int kStage = 65536 + 8192;
-  static constexpr int kP = kLinStages * kStage;         // P: 2 atoms x [128 x 128 B]
-  static constexpr int kVp = kP + 32768;                 // V': 128 rows x 64 B
+  static constexpr int kStage = 65536;
+  static constexpr int kV = kLinStages * kStage;         // [2] x V slice, 128 rows x 64 B (SW64)
+  static constexpr int kVp = kV + 2 * 8192;              // V': 128 rows x 64 B
   static constexpr int kS = kVp + 8192;                  // S bf16: 2 buffers x 128 rows x 64 B
   static constexpr int kPw = kS + 2 * 8192;              // lam^m, m = 0..128
   static constexpr int kBar = kPw + 4 * 132;
-  // ld_full[S], ld_empty[S], qk_full[2], qk_empty[2], ds_full[2], ds_empty[2],
-  // o_full[2], o_empty[2], s_full[2], s_empty[2], vp_full, vp_empty, p_full, p_empty, fin
-  static constexpr int kNumBars = 2 * kLinStages + 12 + 5;
+  // ld_full[S], ld_empty[S], v_full[2], v_empty[2], qk_full[2], qk_empty[2], ds_full[2],
+  // ds_empty[2], o_full[2], o_empty[2], s_full[2], s_empty[2], vp_full, vp_empty, p_full,
+  // p_empty, fin
+  static constexpr int kNumBars = 2 * kLinStages + 4 + 12 + 5;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kTmemCols = 512;
@@ -58,6 +59,7 @@ struct LinTcLayout {
   static constexpr int col_ds(int x) { return 256 + 32 * x; }
   static constexpr int col_oi(int x) { return 320 + 32 * x; }
   static constexpr int col_oe(int x) { return 384 + 32 * x; }
+  static constexpr int kColP = 448;     // P (bf16 pairs): 128 keys in 64 columns, A of P V
 };
 
 // Warps that build the P chunks of each tile: warp w (TMEM lane quadrant
@@ -118,7 +120,9 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* ld_full = bars;
   uint64_t* ld_empty = bars + kLinStages;
-  uint64_t* qk_full = bars + 2 * kLinStages;   // [2]
+  uint64_t* v_full = bars + 2 * kLinStages;    // [2]
+  uint64_t* v_empty = v_full + 2;              // [2]
+  uint64_t* qk_full = v_full + 4;              // [2]
   uint64_t* qk_empty = qk_full + 2;            // [2]
   uint64_t* ds_full = qk_full + 4;             // [2]
   uint64_t* ds_empty = qk_full + 6;            // [2]
@@ -148,6 +152,8 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::mbar_init(ld_empty + s, 1);
     }
     for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(v_full + x, 1);
+      tc::mbar_init(v_empty + x, 1);
       tc::mbar_init(qk_full + x, 1);
       tc::mbar_init(qk_empty + x, kPWarps);
       tc::mbar_init(ds_full + x, 1);
@@ -190,7 +196,10 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
           tc::tma_load_2d(stage + L::kQ + a * 16384, &qmap, ld_full + st, h * D + 64 * a, row0);
           tc::tma_load_2d(stage + L::kK + a * 16384, &kmap, ld_full + st, h * D + 64 * a, row0);
         }
-        tc::tma_load_2d(stage + L::kV, &vmap, ld_full + st, h * D + col0, row0);
+        const int vs = c & 1;
+        if (c >= 2 && !tc::mbar_wait(v_empty + vs, ((c >> 1) - 1) & 1)) break;
+        tc::mbar_expect_tx(v_full + vs, 8192);
+        tc::tma_load_2d(smem + L::kV + vs * 8192, &vmap, v_full + vs, h * D + col0, row0);
       }
     }
   } else if (warp == 1) {
@@ -224,7 +233,7 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         const int st = c % kLinStages, x = c & 1;
         const uint32_t prev = ((c >> 1) - 1) & 1;     // parity of this buffer's previous use
         const uint32_t q = stage_addr(c) + L::kQ, k = stage_addr(c) + L::kK,
-                       v = stage_addr(c) + L::kV;
+                       v = base + L::kV + x * 8192;
         // dS = K^T V'  (A = K^ read MN-major, B = V' MN-major)
         if (!(ok = tc::mbar_wait(vp_full, c & 1))) break;
         if (c >= 2 && !(ok = tc::mbar_wait(ds_empty + x, prev))) break;
@@ -247,112 +256,88 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                           tc::smem_desc_sw64(sb + kk * 1024, 8192, 512), id_o, kk > 0);
         }
         tc::mma_commit(s_empty + x);
+        tc::mma_commit(ld_empty + st);        // Q^ / K^ of tile c are no longer read
         if (c + 1 < n_tiles && !(ok = issue_qk(c + 1))) break;
-        // O_intra = P V
+        // O_intra = P V  (P from TMEM)
         if (!(ok = tc::mbar_wait(p_full, c & 1))) break;
+        if (!(ok = tc::mbar_wait(v_full + x, (c >> 1) & 1))) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::mma_bf16_ss(tmem + L::col_oi(x), tc::smem_desc_sw128(base + L::kP + off, 16, 1024),
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16_ts(tmem + L::col_oi(x), tmem + L::kColP + kk * 8,
                           tc::smem_desc_sw64(v + kk * 1024, 8192, 512), id_o, kk > 0);
-        }
         tc::mma_commit(p_empty);
         tc::mma_commit(o_full + x);
-        tc::mma_commit(ld_empty + st);
+        tc::mma_commit(v_empty + x);
       }
       tc::mma_commit(fin);
       tc::mbar_wait(fin, 0);
     }
   }
 
-  if ((warp >= 2 && warp < 8) && warp != 1) {
-    // ------------------------------------------------------------ V' (warps 4-7) and P
+  if (warp >= 2 && warp < 8) {
+    // ------------------------------------------------------------ P (warps 2-7)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     int clo, chi;
     p_chunks(warp, clo, chi);
-    uint8_t* sP = smem + L::kP;
-    uint8_t* sVp = smem + L::kVp;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     bool ok = true;
     for (int c = 0; ok && c < n_tiles; ++c) {
-      const int st = c % kLinStages, x = c & 1;
-      if (warp >= 4) {
-        // V'_r = lam^(L-1-r) v_r (0 past the end of the sequence)
-        const int Lv = min(kLinTile, N - c * kLinTile);
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + st, (c / kLinStages) & 1));
-        if (ok && c > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(vp_empty, (c - 1) & 1));
-        if (!ok) break;
-        float vv[32];
-        sw64_load_row(smem + st * L::kStage + L::kV, r, vv);
-        const float f = r < Lv ? pw[Lv - 1 - r] : 0.f;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) vv[e] *= f;
-        sw64_store_row(sVp, r, vv);
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(vp_full);
-      }
+      const int x = c & 1;
       // P_rj = QK_rj lam^(r-j) for j <= r (rows past the end are never stored)
       ok = __all_sync(0xffffffffu, tc::mbar_wait(qk_full + x, (c >> 1) & 1));
       if (ok && c > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(p_empty, (c - 1) & 1));
       if (!ok) break;
       tc::tc_fence_after();
-      const uint32_t qk_addr = tmem + ((uint32_t)(quad * 32) << 16) + L::col_qk(x);
-      for (int q0 = clo; q0 < chi; ++q0) {
-        float xv[32];
-        tc::tmem_ld32(qk_addr + 32 * q0, xv);
-        tc::tmem_wait_ld();
+      // both chunk loads are in flight before the single wait
+      float xv[2][32];
+      tc::tmem_ld32(lane_base + L::col_qk(x) + 32 * clo, xv[0]);
+      if (chi - clo > 1) tc::tmem_ld32(lane_base + L::col_qk(x) + 32 * (clo + 1), xv[1]);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int q0 = clo + u;
+        if (q0 >= chi) break;
         if (q0 == quad) {
           // diagonal chunk: column e of the chunk is visible iff e <= lane
 #pragma unroll
-          for (int e = 0; e < 32; ++e) xv[e] = e <= lane ? xv[e] * pw[lane - e] : 0.f;
+          for (int e = 0; e < 32; ++e) xv[u][e] = e <= lane ? xv[u][e] * pw[lane - e] : 0.f;
         } else {
           // below the diagonal: decay lam^(r - 32 q0 - e), applied from e = 31 down
           float dcy = pw[r - 32 * q0 - 31];
 #pragma unroll
           for (int e = 31; e >= 0; --e) {
-            xv[e] *= dcy;
+            xv[u][e] *= dcy;
             dcy *= lam;
           }
         }
-        uint8_t* row = sP + (q0 >> 1) * 16384 + r * 128;
+        uint32_t pk[16];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint4 u;
-          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            h2[e] = __floats2bfloat162_rn(xv[ch * 8 + 2 * e], xv[ch * 8 + 2 * e + 1]);
-          const int chunk = (q0 & 1) * 4 + ch;
-          *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) = u;
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(xv[u][2 * e], xv[u][2 * e + 1]);
+          pk[e] = *reinterpret_cast<uint32_t*>(&h2);
         }
+        tc::tmem_st16_u(lane_base + L::kColP + 16 * q0, pk);
       }
-      // chunks above the diagonal are zero: written once per buffer by the
-      // diagonal owner (warps 4-7) on the first tile, never touched again
-      if (c == 0 && warp >= 4) {
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        for (int q0 = quad + 1; q0 < 4; ++q0) {
-          uint8_t* row = sP + (q0 >> 1) * 16384 + r * 128;
+      if (c == 0 && warp >= 4) {          // chunks above the diagonal stay zero
+        uint32_t z[16];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int chunk = (q0 & 1) * 4 + ch;
-            *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) = z;
-          }
-        }
+        for (int e = 0; e < 16; ++e) z[e] = 0u;
+        for (int q0 = quad + 1; q0 < 4; ++q0) tc::tmem_st16_u(lane_base + L::kColP + 16 * q0, z);
       }
+      tc::tmem_wait_st();
       tc::tc_fence_before();
-      tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         tc::mbar_arrive(qk_empty + x);
         tc::mbar_arrive(p_full);
       }
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ state + epilogue
+  } else if (warp >= 8 && warp < 12) {
+    // ------------------------------------------------------------ state and V'
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;     // key-dim row of S; token row of O
+    const int r = quad * 32 + lane;     // key-dim row of S; token row of V'
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const long long sbase = (((long long)b * H + h) * D + r) * D + col0;
     float S[32];
@@ -362,17 +347,24 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     tc::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(s_full);
-    // gate rows are fetched one tile ahead into registers
-    float gv[32];
-    auto fetch_gate = [&](int c) {
-      const long long off = (((long long)b * N + (long long)c * kLinTile + r) * H + h) * D + col0;
-      if (c < n_tiles && c * kLinTile + r < N) {
+    // V'_r = lam^(L-1-r) v_r of tile c (0 past the end of the sequence)
+    auto make_vp = [&](int c) -> bool {
+      const int Lv = min(kLinTile, N - c * kLinTile);
+      bool okv = __all_sync(0xffffffffu, tc::mbar_wait(v_full + (c & 1), (c >> 1) & 1));
+      if (okv && c > 0) okv = __all_sync(0xffffffffu, tc::mbar_wait(vp_empty, (c - 1) & 1));
+      if (!okv) return false;
+      float vv[32];
+      sw64_load_row(smem + L::kV + (c & 1) * 8192, r, vv);
+      const float f = r < Lv ? pw[Lv - 1 - r] : 0.f;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) load8(gate + off + e, gv + e);
-      }
+      for (int e = 0; e < 32; ++e) vv[e] *= f;
+      sw64_store_row(smem + L::kVp, r, vv);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(vp_full);
+      return true;
     };
-    fetch_gate(0);
-    bool ok = true;
+    bool ok = n_tiles > 0 && make_vp(0);
     for (int c = 0; ok && c < n_tiles; ++c) {
       const int Lv = min(kLinTile, N - c * kLinTile), x = c & 1;
       // S_c = lam^L S_{c-1} + dS
@@ -395,32 +387,56 @@ linear_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_full + buf);
-      // epilogue of tile c: row r = token
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(o_full + x, (c >> 1) & 1));
-      if (!ok) break;
-      tc::tc_fence_after();
-      float oi[32], oe[32];
-      tc::tmem_ld32(lane_base + L::col_oi(x), oi);
-      tc::tmem_ld32(lane_base + L::col_oe(x), oe);
-      tc::tmem_wait_ld();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(o_empty + x);
-      if (r < Lv) {
-        const long long off = (((long long)b * N + (long long)c * kLinTile + r) * H + h) * D + col0;
-        const float fi = pw[r + 1] * scale;
-        float res[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) res[e] = sigmoidf_(gv[e]) * fmaf(fi, oe[e], scale * oi[e]);
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) store8(out + off + e, res + e);
-      }
-      fetch_gate(c + 1);
+      if (c + 1 < n_tiles && !(ok = make_vp(c + 1))) break;
     }
     if (ok && state_out) {
 #pragma unroll
       for (int e = 0; e < 32; e += 4)
         *reinterpret_cast<float4*>(state_out + sbase + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ gated epilogue
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;     // token row of O
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    // gate rows are fetched one tile ahead as raw 16-byte words (converted at
+    // use, so the load latency overlaps the previous tile)
+    constexpr int kGW = 32 * (int)sizeof(T) / 16;
+    uint4 graw[kGW];
+    auto fetch_gate = [&](int c) {
+      const long long off = (((long long)b * N + (long long)c * kLinTile + r) * H + h) * D + col0;
+      if (c < n_tiles && c * kLinTile + r < N) {
+        const uint4* src = reinterpret_cast<const uint4*>(gate + off);
+#pragma unroll
+        for (int e = 0; e < kGW; ++e) graw[e] = src[e];
+      }
+    };
+    fetch_gate(0);
+    const float fs = scale;
+    for (int c = 0; c < n_tiles; ++c) {
+      const int Lv = min(kLinTile, N - c * kLinTile), x = c & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(o_full + x, (c >> 1) & 1))) break;
+      tc::tc_fence_after();
+      const long long off = (((long long)b * N + (long long)c * kLinTile + r) * H + h) * D + col0;
+      const float fi = pw[r + 1] * fs;
+      float gv[32];
+#pragma unroll
+      for (int e = 0; e < 32; e += 8)
+        load8(reinterpret_cast<const T*>(graw) + e, gv + e);
+      float oi[32], oe[32];
+      tc::tmem_ld32(lane_base + L::col_oi(x), oi);
+      tc::tmem_ld32(lane_base + L::col_oe(x), oe);
+      tc::tmem_wait_ld();
+      if (r < Lv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) oi[e] = sigmoidf_(gv[e]) * fmaf(fi, oe[e], fs * oi[e]);
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) store8(out + off + e, oi + e);
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(o_empty + x);
+      fetch_gate(c + 1);
     }
   }
 
