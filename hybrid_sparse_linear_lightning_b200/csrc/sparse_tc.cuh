@@ -30,7 +30,7 @@
 namespace sala {
 
 constexpr int kSpTcThreads = 384;
-constexpr int kSpTcStages = 3;
+constexpr int kSpTcStages = 4;
 constexpr int kSpTcHeadsPerCta = 4;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
@@ -39,19 +39,18 @@ struct SpTcLayout {
   static constexpr int kAtoms = D / 64;                 // 128-byte column atoms of a row
   static constexpr int kQTile = 128 * D * 2;            // one 128-row Q tile
   static constexpr int kKV = 64 * D * 2;                // one 64-row K or V block
-  static constexpr int kP = 128 * 64 * 2;               // one P tile
   static constexpr int kQ = 0;
   static constexpr int kKVBase = kQ + 2 * kQTile;
-  static constexpr int kPBase = kKVBase + kSpTcStages * 2 * kKV;
-  static constexpr int kBar = kPBase + 2 * kP;
+  static constexpr int kBar = kKVBase + kSpTcStages * 2 * kKV;
   // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_done[2], fin
   static constexpr int kNumBars = 1 + 2 * kSpTcStages + 8 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kSel = kMisc + 16;               // int sel[width]
   static constexpr int kBytes(int width) { return kSel + 4 * width; }
-  static constexpr int kTmemCols = D == 128 ? 512 : 256;
-  // TMEM columns: S_0, S_1 (64 each), O_0, O_1 (D each)
+  static constexpr int kTmemCols = 512;
+  // TMEM columns: S_0, S_1 (64 fp32 each), O_0, O_1 (D each), P_0, P_1 (64 bf16 = 32 each)
   static constexpr int kColS0 = 0, kColS1 = 64, kColO0 = 128, kColO1 = 128 + D;
+  static constexpr int kColP0 = 128 + 2 * D, kColP1 = kColP0 + 32;
 };
 
 template <typename T, int D>
@@ -127,7 +126,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
 
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sKV = smem + L::kKVBase;
-  uint8_t* sP = smem + L::kPBase;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -160,8 +158,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     if (tc::elect_one() && n_sel > 0) {
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = tc::smem_u32(sQ), kv_addr = tc::smem_u32(sKV),
-                     p_addr = tc::smem_u32(sP);
+      const uint32_t q_addr = tc::smem_u32(sQ), kv_addr = tc::smem_u32(sKV);
       // Issue order: S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...  so the
       // softmax of one tile overlaps the tensor work of the other.
       auto issue_s = [&](int t, int j) {
@@ -179,9 +176,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         const uint32_t v_addr = kv_addr + (j % kSpTcStages) * 2 * L::kKV + L::kKV;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = tc::smem_desc_sw128(p_addr + t * L::kP + kk * 32, 16, 1024);
           const uint64_t bd = tc::smem_desc_sw128(v_addr + kk * 2048, 64 * 128, 1024);
-          tc::mma_bf16_ss(tmem + (t ? L::kColO1 : L::kColO0), ad, bd, idesc_o, (j > 0 || kk > 0));
+          tc::mma_bf16_ts(tmem + (t ? L::kColO1 : L::kColO0), tmem + (t ? L::kColP1 : L::kColP0) + kk * 8,
+                          bd, idesc_o, (j > 0 || kk > 0));
         }
         tc::mma_commit(o_done + t);
       };
@@ -219,7 +216,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t s_addr = lane_base + (t ? L::kColS1 : L::kColS0);
     const uint32_t o_addr = lane_base + (t ? L::kColO1 : L::kColO0);
-    uint8_t* p_row = sP + t * L::kP + r * 128;
+    const uint32_t p_addr = lane_base + (t ? L::kColP1 : L::kColP0);
+    const float2 sl2v = make_float2(sl2, sl2);
     float m = -INFINITY, l = 0.f;
     bool ok = n_sel > 0;
     for (int j = 0; ok && j < n_sel; ++j) {
@@ -233,16 +231,19 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_free + t);
-      // causal mask on the diagonal block only (warp-uniform branch); the max
-      // is taken on raw logits and scaled once (sl2 > 0)
+      // causal mask on the diagonal block only (warp-uniform branch)
       if (sel[j] == i) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) x[c] = c > tok ? -INFINITY : x[c];
       }
-      float mx = x[0];
+      // row max as a tree over 8 independent partial maxima, scaled once (sl2 > 0)
+      float mp[8];
 #pragma unroll
-      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
-      mx *= sl2;
+      for (int k = 0; k < 8; ++k) mp[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * sl2;
       if (j == 0) m = mx;
       if (j > 0) {
         ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
@@ -265,24 +266,23 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
           tc::tmem_wait_st();
         }
       }
-      // P = exp2(x - m) as bf16, written in the 128B-swizzled K-major layout
-      float rs = 0.f;
+      // P = 2^(x sl2 - m) packed as bf16 pairs into TMEM; row sum over 4 pair-accumulators
+      const float2 negm = make_float2(-m, -m);
+      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+      uint32_t pk[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = exp2f(fmaf(x[ch * 8 + e], sl2, -m));
-          rs += pv[e];
-        }
-        uint4 u;
-        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) h2[e] = __floats2bfloat162_rn(pv[2 * e], pv[2 * e + 1]);
-        *reinterpret_cast<uint4*>(p_row + ((ch ^ (r & 7)) << 4)) = u;
+      for (int e = 0; e < 32; ++e) {
+        const float2 tt = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sl2v, negm);
+        const float2 pv = make_float2(tc::ex2_approx(tt.x), tc::ex2_approx(tt.y));
+        acc4[e & 3] = __fadd2_rn(acc4[e & 3], pv);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(pv.x, pv.y);
+        pk[e] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      l += rs;
-      tc::fence_proxy_async_smem();
+      tc::tmem_st32_u(p_addr, pk);
+      const float2 s01 = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
+      l += s01.x + s01.y;
+      tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(p_full + t);

@@ -239,6 +239,13 @@ __device__ __forceinline__ void named_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// 2^x on the special-function unit (flush-to-zero for tiny results).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------ descriptors
 
 // Shared memory matrix descriptor, 128-byte swizzle.  `lbo` / `sbo` in bytes.
