@@ -192,6 +192,34 @@ class GroupPrefill:
                 timed_calls.append((name, e0, e1))
 
 
+KERNEL_SOURCES = {
+    "sparse_prefill": "sparse_tc.cuh",
+    "linear_prefill": "linear_tc.cuh",
+    "sparse_select": "select.cuh",
+}
+
+
+def kernel_source_hash(call: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "hybrid_sparse_linear_lightning_b200", "csrc", KERNEL_SOURCES[call])
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def kernel_traffic(workload: str, call: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            tr = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = tr.get(workload, {}).get(call)
+    if not ent or ent.get("source_sha256_16") != kernel_source_hash(call):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws <= 1:
@@ -238,7 +266,7 @@ def cpu_baseline_sample(w: wl.Workload, budget_s: float = 20.0):
         threads = len(os.sched_getaffinity(0))
     ln, sp = w.linear, w.sparse
     f64 = lambda t: t.to(torch.float64).numpy()
-    T = 512 if budget_s < 15 else 1024
+    T = 512 if budget_s < 15 else 4096
     q, k, v, g = (f64(x) for x in wl.layer_inputs(w, 0, "cpu", seqlen=T))
     lam = np.asarray(wl.lam_schedule(ln))
     wt = np.ones(ln.head_dim)
@@ -247,7 +275,7 @@ def cpu_baseline_sample(w: wl.Workload, budget_s: float = 20.0):
     t_lin = (time.perf_counter() - t0) / T
     need = (sp.topk + sp.n_init + sp.n_local) * sp.block
     Ns = max(4096, 2 * need)
-    nq = 2 if budget_s < 15 else 4
+    nq = 2 if budget_s < 15 else 8
     nb = Ns // sp.block
     q, k, v, g = (f64(x) for x in wl.layer_inputs(w, w.n_linear, "cpu", seqlen=Ns))
     t0 = time.perf_counter()
@@ -326,15 +354,7 @@ def run_ours(args):
     for c in calls.values():
         c["share"] = round(c["ms"] * c["launches_per_step"] / tot, 4)
     dom = max(calls, key=lambda n: calls[n]["share"])
-    traffic = None
-    try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            tr = json.load(f)
-        ent = tr.get(args.workload, {}).get(dom)
-        if ent and ent.get("kernel_version") == sala.sala_version():
-            traffic = ent["bytes_per_launch"]
-    except (OSError, ValueError):
-        pass
+    traffic = kernel_traffic(args.workload, dom)
     d = calls[dom]
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
                 "unit": d["unit"], "frac": d["frac"], "traffic": traffic, "kernel": dom,
@@ -344,6 +364,12 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(grp, args, ws)
+
+    dec = None
+    if args.decode_steps > 0:
+        del grp
+        torch.cuda.empty_cache()
+        dec = run_decode(wl.WORKLOADS["group_1m"], args.decode_steps, dev, sala, peaks, ws)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -369,11 +395,91 @@ def run_ours(args):
             "tensor_frac_of_step": round(sparse_attn_flops(w, N) / (ms_per_step / 1e3) / 1e12
                                          / peaks["bf16_tflops_sustained"], 4),
             "e2e": e2e, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
+            "decode": dec,
         }
         print(json.dumps(out), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def decode_bytes(w: wl.Workload, cur_len: int) -> float:
+    """Compulsory HBM bytes of one decode step at cache length cur_len:
+    linear states read + written, the complete blocks' key means read, the
+    selected blocks' keys and values read (dominant terms)."""
+    ln, sp = w.linear, w.sparse
+    st = 2.0 * w.n_linear * w.batch * ln.heads * ln.head_dim * ln.head_dim * 4
+    nb = cur_len // sp.block
+    kb = float(w.batch * nb * sp.kv_heads * sp.head_dim * 4)
+    sel = min(nb + 1, sp.topk + sp.n_init + sp.n_local)
+    kv = float(w.batch * sp.kv_heads * sel * sp.block * sp.head_dim * 2 * 2)
+    return st + kb + kv
+
+
+def run_decode(w: wl.Workload, steps: int, dev, sala, peaks, ws):
+    """Prefill the 1M-token group layer by layer (keeping only the linear
+    states and the sparse layer's key / value caches), then time `steps`
+    decode tokens through the C ABI with CUDA events."""
+    N = w.seqlen
+    ln, sp = w.linear, w.sparse
+    B, H, D = w.batch, ln.heads, ln.head_dim
+    cap = N + ((steps + sp.block - 1) // sp.block + 1) * sp.block
+    lam = torch.tensor(wl.lam_schedule(ln), dtype=torch.float32, device=dev)
+    wt = wl.rms_weights(D, dev)
+    states = []
+    for l in range(w.n_linear):
+        q, k, v, g = wl.layer_inputs(w, l, dev)
+        out, st = sala.linear_prefill(q, k, v, g, lam, wt, wt, chunk=ln.chunk, want_state=True)
+        states.append(st)
+        del q, k, v, g, out
+        torch.cuda.empty_cache()
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev)
+    k_cache = torch.zeros((B, cap, sp.kv_heads, D), dtype=torch.bfloat16, device=dev)
+    v_cache = torch.zeros_like(k_cache)
+    kbar = torch.zeros((B, cap // sp.block, sp.kv_heads, D), dtype=torch.float32, device=dev)
+    ksum = torch.zeros((B, sp.kv_heads, D), dtype=torch.float32, device=dev)
+    qn, kn, kb, idx = sala.sparse_select(q, k, wt, wt, block=sp.block, topk=sp.topk,
+                                         n_init=sp.n_init, n_local=sp.n_local)
+    k_cache[:, :N] = kn
+    v_cache[:, :N] = v
+    kbar[:, :N // sp.block] = kb
+    del q, k, v, g, qn, kn, kb, idx
+    torch.cuda.empty_cache()
+    ld = sala.linear_desc(B, 64, H, D, ln.chunk, w.torch_dtype)
+    sd = sala.sparse_desc(B, 64, sp.q_heads, sp.kv_heads, D, sp.block, sp.topk, sp.n_init,
+                          sp.n_local, w.torch_dtype)
+    dd = sala.DecodeDesc(ld, sd, w.n_linear, cap)
+    wsd = sala.workspace(sala.sala_decode_workspace_size(dd), dev)
+    toks = [wl.decode_inputs(w, s, dev) for s in range(steps + 3)]
+    outs = [torch.empty_like(t[0]) for t in toks[0]]
+    ios = [sala.make_decode_io(t, outs, states, [lam] * w.n_linear, wt, wt) for t in toks]
+
+    def step(s, pos):
+        r = sala.sala_decode_step(dd, ios[s], k_cache, v_cache, kbar, ksum, pos, wsd)
+        if r != 0:
+            raise RuntimeError("decode: " + sala.status_string(r))
+
+    for s in range(3):                       # warm-up tokens
+        step(s, N + s)
+    torch.cuda.synchronize()
+    l0 = sala.sala_kernel_launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(steps):
+        step(s + 3, N + 3 + s)
+    e1.record()
+    torch.cuda.synchronize()
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set during decode")
+    ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    us = ms * 1e3 / steps
+    byts = sum(decode_bytes(w, N + 3 + s) for s in range(steps)) / steps
+    gbs = byts / (us * 1e-6) / 1e9
+    return {"workload": w.name, "context": N, "steps": steps, "us_per_step": round(us, 2),
+            "tokens_per_s": round(ws * 1e6 / us, 1), "bytes_per_step": int(byts),
+            "achieved_GBps": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+            "launches_per_step": (sala.sala_kernel_launch_count() - l0) / steps}
 
 
 def run_e2e(grp: GroupPrefill, args, ws):
@@ -458,6 +564,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--decode-steps", type=int, default=256,
+                    help="decode tokens timed after a 1M-token prefill (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
