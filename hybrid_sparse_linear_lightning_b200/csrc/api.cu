@@ -236,21 +236,32 @@ sala_status run_sparse_prefill(const sala_sparse_desc* d, const void* qn, const 
 }
 
 struct DecodeWs {
-  size_t qhat, qgrp, keys, idx, part, total;
+  size_t qhat, qgrp, cand_key, cand_idx, idx, part, counters, total;
 };
+constexpr int kDecodeMergeMax = 8192;   // candidates entering the exact merge
 DecodeWs decode_ws(const sala_decode_desc* d) {
   const sala_sparse_desc& s = d->sp;
   const size_t B = s.batch, Hq = s.q_heads, Hkv = s.kv_heads, D = s.head_dim;
   const size_t width = s.topk + s.n_init + s.n_local;
-  const size_t capb = (size_t)(d->cache_capacity / s.block);
   DecodeWs w;
   w.qhat = 0;
   w.qgrp = w.qhat + align_up(B * Hq * D * 4);
-  w.keys = w.qgrp + align_up(B * Hkv * D * 4);
-  w.idx = w.keys + align_up(B * Hkv * capb * 4);
+  w.cand_key = w.qgrp + align_up(B * Hkv * D * 4);
+  w.cand_idx = w.cand_key + align_up(B * Hkv * kDecodeMergeMax * 4);
+  w.idx = w.cand_idx + align_up(B * Hkv * kDecodeMergeMax * 4);
   w.part = w.idx + align_up(B * Hkv * width * 4);
-  w.total = w.part + align_up(B * Hkv * width * (Hq / Hkv) * (D + 2) * 4);
+  w.counters = w.part + align_up(B * Hkv * width * (Hq / Hkv) * (D + 4) * 4);
+  w.total = w.counters + align_up(B * Hkv * 2 * 4);
   return w;
+}
+
+// Candidate chunk of the decode selection: 256 blocks, doubled until the
+// local lists (chunks x k) fit the exact merge.
+void decode_chunks(int n_cand, int k, int* chunk, int* n_chunks) {
+  int c = 256;
+  while (k > 0 && (long long)((n_cand + c - 1) / c) * k > kDecodeMergeMax) c *= 2;
+  *chunk = c;
+  *n_chunks = n_cand > 0 ? (n_cand + c - 1) / c : 1;
 }
 
 sala_status check_decode(const sala_decode_desc* d) {
@@ -268,6 +279,7 @@ sala_status check_decode(const sala_decode_desc* d) {
   if (d->lin.batch != d->sp.batch || d->lin.dtype != d->sp.dtype) return SALA_ERR_INVALID_ARG;
   if (d->cache_capacity < d->sp.block || d->cache_capacity % d->sp.block != 0) return SALA_ERR_INVALID_ARG;
   if (d->cache_capacity / d->sp.block > 49152) return SALA_ERR_UNSUPPORTED;
+  if (d->sp.q_heads > kDecodeMaxQHeads) return SALA_ERR_UNSUPPORTED;
   return SALA_OK;
 }
 
@@ -275,7 +287,12 @@ template <typename T, int DL, int DS>
 sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void* k_cache,
                        void* v_cache, float* kbar, float* ksum, int64_t cur_len, char* ws,
                        cudaStream_t st) {
+  static_assert(DL == DS, "one head_dim for the group");
+  constexpr int D = DS;
   const sala_linear_desc& L = d->lin;
+  const sala_sparse_desc& S = d->sp;
+  const int sl = d->n_linear;
+  const DecodeWs w = decode_ws(d);
   DecodeLinearArgs a;
   memset(&a, 0, sizeof(a));
   for (int l = 0; l < d->n_linear; ++l) {
@@ -283,49 +300,46 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
     a.wq[l] = io->wq[l]; a.wk[l] = io->wk[l]; a.lambda[l] = io->lambda[l];
     a.state[l] = io->lin_state[l]; a.out[l] = io->out[l];
   }
-  decode_linear_kernel<T, DL><<<d->n_linear * L.batch * L.heads * (DL / 64), 256, 0, st>>>(
-      a, L.batch, L.heads, cur_len, log2((double)L.rope_base), L.rms_eps, L.scale);
+  DecodeSparseArgs sp;
+  sp.q = io->q[sl]; sp.k = io->k[sl]; sp.v = io->v[sl]; sp.wq = io->wq[sl]; sp.wk = io->wk[sl];
+  sp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  sp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  sp.kbar = kbar;
+  sp.ksum = ksum;
+  sp.qhat = reinterpret_cast<float*>(ws + w.qhat);
+  sp.qgrp = reinterpret_cast<float*>(ws + w.qgrp);
+  sp.counters = reinterpret_cast<unsigned*>(ws + w.counters);
+  // 1. linear layers + sparse prep
+  const int n_lin = d->n_linear * L.batch * L.heads * (D / 64);
+  decode_stage1_kernel<T, D><<<n_lin + S.batch, 256, 0, st>>>(
+      a, sp, n_lin, L.batch, L.heads, S.q_heads, S.kv_heads, d->cache_capacity, cur_len, S.block,
+      log2((double)L.rope_base), L.rms_eps, S.rms_eps, L.scale);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-
-  const sala_sparse_desc& S = d->sp;
-  const int sl = d->n_linear;
-  const DecodeWs w = decode_ws(d);
-  float* qhat = reinterpret_cast<float*>(ws + w.qhat);
-  float* qgrp = reinterpret_cast<float*>(ws + w.qgrp);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(ws + w.keys);
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
-  float* part = reinterpret_cast<float*>(ws + w.part);
+  // 2. selection
   const long long capb = d->cache_capacity / S.block;
   const int width = S.topk + S.n_init + S.n_local;
-  decode_sparse_prep_kernel<T, DS><<<S.batch, 256, 0, st>>>(
-      static_cast<const T*>(io->q[sl]), static_cast<const T*>(io->k[sl]),
-      static_cast<const T*>(io->v[sl]), io->wq[sl], io->wk[sl],
-      static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), kbar, ksum,
-      qhat, qgrp, S.q_heads, S.kv_heads, d->cache_capacity, cur_len, S.block, S.rms_eps);
-  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
   const int bcur = (int)(cur_len / S.block);
   const int n_cand = std::max(0, bcur - S.n_local + 1 - S.n_init);
-  if (n_cand > S.topk) {
-    const long long total = (long long)S.batch * S.kv_heads * n_cand;
-    decode_scores_kernel<DS><<<(unsigned)((total + 7) / 8), 256, 0, st>>>(
-        qgrp, kbar, keys, S.kv_heads, capb, S.n_init, n_cand, total);
-    if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  }
-  const size_t smem = (size_t)std::max(n_cand, 1) * 4;
-  if (allow_smem(decode_topk_kernel, smem) != cudaSuccess) return SALA_ERR_CUDA;
-  decode_topk_kernel<<<S.batch * S.kv_heads, kSelectThreads, smem, st>>>(
-      keys, idx, S.kv_heads, capb, bcur, S.topk, S.n_init, S.n_local, width);
+  const int k = std::min(S.topk, n_cand);
+  int chunk = 512, n_chunks = 1;
+  if (k > 0 && k < n_cand) decode_chunks(n_cand, k, &chunk, &n_chunks);
+  const size_t sel_smem = (size_t)std::max(2 * chunk, 2 * n_chunks * k + k) * 4;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
+  if (allow_smem(decode_select_kernel<D>, sel_smem) != cudaSuccess) return SALA_ERR_CUDA;
+  decode_select_kernel<D><<<S.batch * S.kv_heads * n_chunks, kSelectThreads, sel_smem, st>>>(
+      sp.qgrp, kbar, reinterpret_cast<uint32_t*>(ws + w.cand_key),
+      reinterpret_cast<int32_t*>(ws + w.cand_idx), idx, sp.counters, S.kv_heads, capb, bcur,
+      S.topk, S.n_init, S.n_local, width, chunk, n_chunks);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  const size_t asmem = sizeof(float) * 64 * (2 * DS + 1);
-  if (allow_smem(decode_attn_kernel<DS>, asmem) != cudaSuccess) return SALA_ERR_CUDA;
-  decode_attn_kernel<DS><<<S.batch * S.kv_heads * width, 256, asmem, st>>>(
-      qhat, static_cast<const __nv_bfloat16*>(k_cache), static_cast<const __nv_bfloat16*>(v_cache),
-      idx, part, S.q_heads, S.kv_heads, d->cache_capacity, cur_len, S.block, width,
-      sparse_scale(&S));
-  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  decode_combine_kernel<T, DS><<<S.batch * S.q_heads, DS, 0, st>>>(
-      part, static_cast<const T*>(io->gate[sl]), static_cast<T*>(io->out[sl]), S.q_heads,
-      S.kv_heads, width);
+  // 3. attention partials, combine and gate
+  const int G = S.q_heads / S.kv_heads;
+  const size_t att_smem = std::max((size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 + G * 8,
+                                   ((size_t)2 * width * G + G) * 4);   // staging of the combine
+  if (allow_smem(decode_attn_kernel<T, D>, att_smem) != cudaSuccess) return SALA_ERR_CUDA;
+  decode_attn_kernel<T, D><<<S.batch * S.kv_heads * width, 256, att_smem, st>>>(
+      sp.qhat, sp.k_cache, sp.v_cache, idx, reinterpret_cast<float*>(ws + w.part), sp.counters,
+      static_cast<const T*>(io->gate[sl]), static_cast<T*>(io->out[sl]), S.q_heads, S.kv_heads,
+      d->cache_capacity, cur_len, S.block, width, sparse_scale(&S) * 1.4426950408889634f);
   return launch_status();
 }
 

@@ -67,14 +67,30 @@ __device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_can
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, bin = 0;
-      for (bin = 255; bin >= 0; --bin) {
-        if (cum + hist[bin] >= need) break;
-        cum += hist[bin];
+    if (tid < 32) {
+      // bins from the top: lane l owns bins 255 - 8l .. 248 - 8l; find the bin
+      // where the count of larger-or-equal keys first reaches `need`
+      const int lane = tid;
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { cnt[u] = hist[255 - 8 * lane - u]; tot += cnt[u]; }
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      *s_prefix = prefix | ((uint32_t)bin << shift);
-      *s_need = need - cum;
+      const int before = incl - tot;
+      const unsigned hit = __ballot_sync(0xffffffffu, before < need && incl >= need);
+      if (lane == __ffs(hit) - 1) {
+        int cum = before, u = 0;
+        for (; u < 8; ++u) {
+          if (cum + cnt[u] >= need) break;
+          cum += cnt[u];
+        }
+        *s_prefix = prefix | ((uint32_t)(255 - 8 * lane - u) << shift);
+        *s_need = need - cum;
+      }
     }
     __syncthreads();
     prefix = *s_prefix;
