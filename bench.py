@@ -241,12 +241,20 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank time over all ranks (device tensor under NCCL, host
+    tensor under gloo)."""
     if ws <= 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(tokens_per_rank_step: int, steps: int, max_ms: float, ws: int) -> float:
+    """Whole-job tokens/s of `ws` independent replicas timed by the slowest."""
+    return tokens_per_rank_step * ws * steps / (max_ms / 1e3)
 
 
 def cpu_baseline_sample(w: wl.Workload, budget_s: float = 20.0):
@@ -330,8 +338,7 @@ def run_ours(args):
     for name, e0, e1 in timed:
         per_call.setdefault(name, []).append(e0.elapsed_time(e1))
     ms_per_step = elapsed_ms / args.steps
-    tokens = w.batch * N * ws * args.steps
-    value = tokens / (elapsed_ms / 1e3)
+    value = replica_throughput(w.batch * N, args.steps, elapsed_ms, ws)
 
     # per-call roofline (dominant call reported as "roofline")
     calls = {}
