@@ -194,16 +194,26 @@ class GroupPrefill:
 
 KERNEL_SOURCES = {
     "sparse_prefill": "sparse_tc.cuh",
-    "linear_prefill": "linear_tc.cuh",
+    "linear_prefill": "linear_seg_tc.cuh",
     "sparse_select": "select.cuh",
 }
 
 
-def kernel_source_hash(call: str) -> str:
+def code_hash(text: str) -> str:
+    """Hash of a CUDA source with comments removed and whitespace collapsed,
+    so that edits to comments alone keep stored counters valid."""
     import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
+def kernel_source_hash(call: str) -> str:
     path = os.path.join(ROOT, "hybrid_sparse_linear_lightning_b200", "csrc", KERNEL_SOURCES[call])
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path, encoding="utf-8") as f:
+        return code_hash(f.read())
 
 
 def kernel_traffic(workload: str, call: str):

@@ -15,7 +15,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "linear_simt.cuh"
-#include "linear_tc.cuh"
+#include "linear_seg_tc.cuh"
 #include "prologue.cuh"
 #include "select.cuh"
 #include "sparse_simt.cuh"
@@ -76,21 +76,29 @@ inline float sparse_scale(const sala_sparse_desc* d) {
 }
 
 struct LinearWs {
-  size_t qn, kn, total;
+  size_t qn, kn, seg, total;
 };
+inline bool linear_on_tc(const sala_linear_desc* d) {
+  return d->dtype == SALA_BF16 && d->head_dim == 128;
+}
 LinearWs linear_ws(const sala_linear_desc* d) {
   const size_t n = (size_t)d->batch * d->seqlen * d->heads * d->head_dim;
   LinearWs w;
   w.qn = 0;
   w.kn = align_up(n * 2);
-  w.total = w.kn + align_up(n * 2);
+  w.seg = w.kn + align_up(n * 2);
+  w.total = w.seg;
+  if (linear_on_tc(d)) {
+    const LinSegPlan p = lin_seg_plan(d->batch, d->heads, d->seqlen);
+    w.total += align_up((size_t)d->batch * d->heads * p.n_seg * 128 * 128 * 4);
+  }
   return w;
 }
 
-sala_status run_linear_tc(const sala_linear_desc* d, const __nv_bfloat16* qn,
-                          const __nv_bfloat16* kn, const void* v, const void* gate,
-                          const float* lambda, const float* state_in, float* state_out, void* out,
-                          cudaStream_t st);
+sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
+                           const __nv_bfloat16* kn, const void* v, const void* gate,
+                           const float* lambda, const float* state_in, float* state_out,
+                           void* out, float* seg_state, cudaStream_t st);
 
 template <typename T, int D>
 sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, const void* v,
@@ -109,7 +117,8 @@ sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, 
   // bf16 activations with head_dim 128 run on the tensor cores; fp32
   // activations and head_dim 64 on CUDA cores.
   if (std::is_same<T, __nv_bfloat16>::value && D == 128)
-    return run_linear_tc(d, qn, kn, v, gate, lambda, state_in, state_out, out, st);
+    return run_linear_seg(d, qn, kn, v, gate, lambda, state_in, state_out, out,
+                          reinterpret_cast<float*>(ws + w.seg), st);
   const size_t smem = sizeof(SimtSmem<D>);
   if (allow_smem(linear_chunk_simt_kernel<T, D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
   const int grid = d->batch * d->heads * (D / kSimtCols);
@@ -171,25 +180,43 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-sala_status run_linear_tc(const sala_linear_desc* d, const __nv_bfloat16* qn,
-                          const __nv_bfloat16* kn, const void* v, const void* gate,
-                          const float* lambda, const float* state_in, float* state_out, void* out,
-                          cudaStream_t st) {
+sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
+                           const __nv_bfloat16* kn, const void* v, const void* gate,
+                           const float* lambda, const float* state_in, float* state_out,
+                           void* out, float* seg_state, cudaStream_t st) {
   constexpr int D = 128;
+  const LinSegPlan p = lin_seg_plan(d->batch, d->heads, d->seqlen);
   const uint64_t rows = (uint64_t)d->batch * d->seqlen, cols = (uint64_t)d->heads * D;
-  CUtensorMap qm, km, vm;
-  if (!make_tmap_bf16(&qm, qn, cols, rows, 64, kLinTile) ||
-      !make_tmap_bf16(&km, kn, cols, rows, 64, kLinTile) ||
-      !make_tmap_bf16(&vm, v, cols, rows, kLinCols, kLinTile, CU_TENSOR_MAP_SWIZZLE_64B))
+  CUtensorMap qm, km, vm, gm;
+  if (!make_tmap_bf16(&qm, qn, cols, rows, 64, kLsTile) ||
+      !make_tmap_bf16(&km, kn, cols, rows, 64, kLsTile) ||
+      !make_tmap_bf16(&vm, v, cols, rows, 64, kLsTile) ||
+      !make_tmap_bf16(&gm, gate, cols, rows, 64, kLsTile))
     return SALA_ERR_CUDA;
-  const size_t smem = LinTcLayout::kBytes + 1024;
-  auto kern = linear_attn_tc_kernel<__nv_bfloat16>;
-  if (allow_smem(kern, smem) != cudaSuccess) return SALA_ERR_CUDA;
-  const int grid = d->batch * d->heads * (D / kLinCols);
-  kern<<<grid, kLinTcThreads, smem, st>>>(qm, km, vm, static_cast<const __nv_bfloat16*>(gate),
-                                          lambda, state_in, state_out,
-                                          static_cast<__nv_bfloat16*>(out), d->seqlen, d->heads,
-                                          d->scale);
+  const int grid = d->batch * d->heads * p.n_seg;
+  // 1. segment sums
+  const size_t smem_a = LsSumLayout::kBytes + 1024;
+  if (allow_smem(linear_segsum_kernel, smem_a) != cudaSuccess) return SALA_ERR_CUDA;
+  linear_segsum_kernel<<<grid, kLsSumThreads, smem_a, st>>>(km, vm, lambda, seg_state, d->seqlen,
+                                                            d->heads, p.seg_tiles, p.n_seg);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  // 2. scan over segments
+  const long long n_el = (long long)d->batch * d->heads * D * D;
+  linear_segscan_kernel<<<(unsigned)((n_el + kLsScanThreads - 1) / kLsScanThreads), kLsScanThreads,
+                          0, st>>>(lambda, state_in, state_out, seg_state, d->seqlen, d->heads,
+                                   p.seg_tiles, p.n_seg, n_el);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  // 3. outputs
+  const size_t smem_b = LsOutLayout::kBytes + 1024;
+  auto kern = linear_segout_kernel<__nv_bfloat16>;
+  if (allow_smem(kern, smem_b) != cudaSuccess) return SALA_ERR_CUDA;
+  // the in-kernel register split assumes this launch allocation exactly
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SALA_ERR_CUDA;
+  if (fa.numRegs != kLsOutRegsLaunch) return SALA_ERR_UNSUPPORTED;
+  kern<<<grid, kLsOutThreads, smem_b, st>>>(qm, km, vm, gm, static_cast<const __nv_bfloat16*>(gate),
+                                            lambda, seg_state, static_cast<__nv_bfloat16*>(out),
+                                            d->seqlen, d->heads, p.seg_tiles, p.n_seg, d->scale);
   return launch_status();
 }
 

@@ -73,6 +73,15 @@ __device__ __forceinline__ float warp_max(float x) {
 // ulp; the outputs are rounded to bf16 or checked at 1e-2).
 __device__ __forceinline__ float sigmoidf_(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
+// Logistic sigmoid as 1/2 + tanh(x/2)/2 on the hardware tanh approximation
+// (one special-function op; absolute error about 2^-11, below the bf16
+// rounding of the outputs it scales).
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
+
 // Order-preserving map of an fp32 score to uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t score_key(float s) {
   uint32_t u = __float_as_uint(s);

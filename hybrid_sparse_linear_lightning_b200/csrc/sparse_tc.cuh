@@ -11,8 +11,8 @@
 // Per selected block j (64 keys):  S_t = Q_t K_j^T  (tcgen05, M=128 N=64,
 // fp32 in TMEM);  softmax warps read S_t one row per thread, apply the causal
 // mask on the diagonal block, exponentiate against a running max, write
-// P_t (bf16) to shared memory;  O_t += P_t V_j  (tcgen05, M=128 N=d, fp32 in
-// TMEM).  Exact softmax: the running max is raised (and O, l rescaled) only
+// P_t (bf16 pairs) back to TMEM;  O_t += P_t V_j  (tcgen05 with A read from
+// TMEM, M=128 N=d, fp32 in TMEM).  Exact softmax: the running max is raised (and O, l rescaled) only
 // when a row's max grows by more than 2^8, so values stay bounded; the final
 // division by l makes the result independent of that choice up to rounding.
 // Epilogue: out = sigmoid(gate) * O / l.

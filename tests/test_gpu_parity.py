@@ -61,6 +61,30 @@ def test_linear_bf16_d128(sala, lam_kind, seqlen):
     assert rel_err(f64(st), S) <= TOL
 
 
+def test_linear_batch2_multi_tile_segments(sala):
+    """Batch 2 x 32 heads at 7360 tokens: each sequence splits into segments
+    of four 128-token tiles (the last of two tiles, ending on a 64-token
+    tile), with a state carried in.  Heads 0, 7 and 31: outputs and final
+    states."""
+    dev = torch.device("cuda")
+    w = _w("group_32k", batch=2)
+    N = 7360
+    q, k, v, g = wl.layer_inputs(w, 0, dev, seqlen=N)
+    lam = lam_tensor(w, dev)
+    wq = wl.rms_weights(128, dev)
+    gen = torch.Generator(device=dev).manual_seed(7)
+    s_in = 0.05 * torch.randn((2, 32, 128, 128), generator=gen, device=dev)
+    out, st = sala.linear_prefill(q, k, v, g, lam, wq, wq, pos0=3, state_in=s_in, want_state=True)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    heads = [0, 7, 31]
+    sub = lambda t: f64(t[:, :, heads])
+    ref, S = oracle.linear_layer(sub(q), sub(k), sub(v), sub(g), f64(lam)[heads], f64(wq), f64(wq),
+                                 pos0=3, state_in=f64(s_in[:, heads]))
+    assert rel_err(sub(out), ref) <= TOL
+    assert rel_err(f64(st[:, heads]), S) <= TOL
+
+
 def test_linear_special_lambdas(sala):
     dev = torch.device("cuda")
     w = _w("group_32k")
