@@ -263,7 +263,7 @@ sala_status run_sparse_prefill(const sala_sparse_desc* d, const void* qn, const 
 }
 
 struct DecodeWs {
-  size_t qhat, qgrp, cand_key, cand_idx, idx, part, counters, total;
+  size_t qhat, cand_key, cand_idx, idx, part, counters, total;
 };
 constexpr int kDecodeMergeMax = 8192;   // candidates entering the exact merge
 DecodeWs decode_ws(const sala_decode_desc* d) {
@@ -272,8 +272,7 @@ DecodeWs decode_ws(const sala_decode_desc* d) {
   const size_t width = s.topk + s.n_init + s.n_local;
   DecodeWs w;
   w.qhat = 0;
-  w.qgrp = w.qhat + align_up(B * Hq * D * 4);
-  w.cand_key = w.qgrp + align_up(B * Hkv * D * 4);
+  w.cand_key = w.qhat + align_up(B * Hq * D * 4);
   w.cand_idx = w.cand_key + align_up(B * Hkv * kDecodeMergeMax * 4);
   w.idx = w.cand_idx + align_up(B * Hkv * kDecodeMergeMax * 4);
   w.part = w.idx + align_up(B * Hkv * width * 4);
@@ -334,13 +333,17 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   sp.kbar = kbar;
   sp.ksum = ksum;
   sp.qhat = reinterpret_cast<float*>(ws + w.qhat);
-  sp.qgrp = reinterpret_cast<float*>(ws + w.qgrp);
   sp.counters = reinterpret_cast<unsigned*>(ws + w.counters);
   // 1. linear layers + sparse prep
+  RopeFreq rf;
+  memset(&rf, 0, sizeof(rf));
+  const double log2_base = log2((double)L.rope_base);
+  for (int i = 0; i < D / 2; ++i) rf.inv[i] = exp2(-2.0 * i / D * log2_base);
   const int n_lin = d->n_linear * L.batch * L.heads * (D / 64);
-  decode_stage1_kernel<T, D><<<n_lin + S.batch, 256, 0, st>>>(
-      a, sp, n_lin, L.batch, L.heads, S.q_heads, S.kv_heads, d->cache_capacity, cur_len, S.block,
-      log2((double)L.rope_base), L.rms_eps, S.rms_eps, L.scale);
+  const int n_sp = (S.kv_heads + S.q_heads + kDecodeRowsPerCta - 1) / kDecodeRowsPerCta;
+  decode_stage1_kernel<T, D><<<n_lin + S.batch * n_sp, 256, 0, st>>>(
+      a, sp, n_lin, n_sp, L.batch, L.heads, S.q_heads, S.kv_heads, d->cache_capacity, cur_len,
+      S.block, rf, L.rms_eps, S.rms_eps, L.scale);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
   // 2. selection
   const long long capb = d->cache_capacity / S.block;
@@ -354,19 +357,28 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
   if (allow_smem(decode_select_kernel<D>, sel_smem) != cudaSuccess) return SALA_ERR_CUDA;
   decode_select_kernel<D><<<S.batch * S.kv_heads * n_chunks, kSelectThreads, sel_smem, st>>>(
-      sp.qgrp, kbar, reinterpret_cast<uint32_t*>(ws + w.cand_key),
-      reinterpret_cast<int32_t*>(ws + w.cand_idx), idx, sp.counters, S.kv_heads, capb, bcur,
+      sp.qhat, kbar, reinterpret_cast<uint32_t*>(ws + w.cand_key),
+      reinterpret_cast<int32_t*>(ws + w.cand_idx), idx, sp.counters, S.q_heads, S.kv_heads, capb, bcur,
       S.topk, S.n_init, S.n_local, width, chunk, n_chunks);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  // 3. attention partials, combine and gate
+  // 3. attention partials
   const int G = S.q_heads / S.kv_heads;
-  const size_t att_smem = std::max((size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 + G * 8,
-                                   ((size_t)2 * width * G + G) * 4);   // staging of the combine
+  const int n_parts = (width + kDecodeBlocksPerCta - 1) / kDecodeBlocksPerCta;
+  // K, V staging + queries + logits + running outputs + (m, l) + factors
+  const size_t att_smem = (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
+                          (size_t)G * D * 4 + (size_t)G * 12;
   if (allow_smem(decode_attn_kernel<T, D>, att_smem) != cudaSuccess) return SALA_ERR_CUDA;
-  decode_attn_kernel<T, D><<<S.batch * S.kv_heads * width, 256, att_smem, st>>>(
-      sp.qhat, sp.k_cache, sp.v_cache, idx, reinterpret_cast<float*>(ws + w.part), sp.counters,
-      static_cast<const T*>(io->gate[sl]), static_cast<T*>(io->out[sl]), S.q_heads, S.kv_heads,
-      d->cache_capacity, cur_len, S.block, width, sparse_scale(&S) * 1.4426950408889634f);
+  float* part = reinterpret_cast<float*>(ws + w.part);
+  decode_attn_kernel<T, D><<<S.batch * S.kv_heads * n_parts, 256, att_smem, st>>>(
+      sp.qhat, sp.k_cache, sp.v_cache, idx, part, S.q_heads, S.kv_heads, d->cache_capacity,
+      cur_len, S.block, width, n_parts, sparse_scale(&S) * 1.4426950408889634f);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  // 4. combine and gate, one CTA per q head
+  const size_t cmb_smem = (size_t)2 * n_parts * 4;
+  if (allow_smem(decode_combine_kernel<T, D>, cmb_smem) != cudaSuccess) return SALA_ERR_CUDA;
+  decode_combine_kernel<T, D><<<S.batch * S.q_heads, D, cmb_smem, st>>>(
+      part, static_cast<const T*>(io->gate[sl]), static_cast<T*>(io->out[sl]), S.q_heads,
+      S.kv_heads, n_parts);
   return launch_status();
 }
 

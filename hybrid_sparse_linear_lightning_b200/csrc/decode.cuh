@@ -11,11 +11,11 @@
 // initial and local blocks (the block holding the token is local), and runs
 // exact softmax attention over them (split over blocks, then combined).
 //
-// Three launches per token: (1) linear-layer state updates and the sparse
+// Four launches per token: (1) linear-layer state updates and the sparse
 // layer's normalisation / cache append in one grid; (2) block scores with a
 // per-chunk top-k, merged exactly by the last CTA of each kv head; (3) one
-// CTA per selected block computing partial softmax sums, combined and gated
-// by the last CTA of each kv head.
+// CTA per selected block computing partial softmax sums; (4) their combine
+// and the gate, one CTA per q head.
 #pragma once
 
 #include "common.cuh"
@@ -47,15 +47,18 @@ struct DecodeSparseArgs {
   float* kbar;
   float* ksum;
   float* qhat;          // [B, Hq, D] normalised queries
-  float* qgrp;          // [B, Hkv, D] group sums
-  unsigned* counters;   // [B, Hkv, 2]: select / attention completion counts
+  unsigned* counters;   // [B, Hkv, 2]: selection completion counts (second unused)
+};
+
+// RoPE inverse frequencies base^(-2i/D), i < D/2, formed in fp64 on the host.
+struct RopeFreq {
+  double inv[64];
 };
 
 // cos / sin of p * base^(-2i/D): the argument is formed and reduced modulo
 // 2 pi in fp64 (|p| < 2^53), then evaluated in fp32 on [-pi, pi].
-__device__ __forceinline__ void rope_cs(long long p, int i, int D, double log2_base, float& c,
-                                        float& s) {
-  const double a = (double)p * exp2(-2.0 * i / D * log2_base);
+__device__ __forceinline__ void rope_cs(long long p, double inv_freq, float& c, float& s) {
+  const double a = (double)p * inv_freq;
   const double two_pi = 6.283185307179586476925286766559;
   const double r = a - rint(a / two_pi) * two_pi;
   sincosf((float)r, &s, &c);
@@ -63,18 +66,19 @@ __device__ __forceinline__ void rope_cs(long long p, int i, int D, double log2_b
 
 // Stage 1.  CTAs [0, n_lin): one per (linear layer, batch, head, 64-column
 // slice) updating S <- lam S + k^T v and writing out = sigmoid(g) q^ S.
-// CTAs [n_lin, n_lin + B): the sparse layer of batch b (normalise k and
-// append it and v to the caches, update the running block sum / mean,
-// normalise q, form the group sums, reset the completion counters).
-constexpr int kDecodeMaxQHeads = 64;   // q heads of the sparse layer handled by stage 1
+// CTAs [n_lin, n_lin + B * n_sp): the sparse layer, one warp per row of the
+// Hkv keys and Hq queries of batch b (normalise k and append it and v to the
+// caches, update the running block sum / mean; normalise q); the first of
+// them also resets the completion counters.
+constexpr int kDecodeMaxQHeads = 64;   // q heads of the sparse layer (selection staging)
+constexpr int kDecodeRowsPerCta = 8;   // sparse-layer rows per stage-1 CTA
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int B, int H, int Hq,
-                     int Hkv, long long cap, long long pos, int BLK, double log2_base, float eps_l,
-                     float eps_s, float scale) {
+decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int n_sp, int B, int H,
+                     int Hq, int Hkv, long long cap, long long pos, int BLK, RopeFreq rf,
+                     float eps_l, float eps_s, float scale) {
   __shared__ float sh[D * 3 + 256];
-  __shared__ float qsm[kDecodeMaxQHeads * D];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if ((int)blockIdx.x < n_lin) {
     constexpr int NSL = D / 64;
@@ -99,7 +103,7 @@ decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int B, 
         const float x1 = to_f32(src[voff + i]) * r * w[i];
         const float x2 = to_f32(src[voff + i + D / 2]) * r * w[i + D / 2];
         float c, s;
-        rope_cs(pos, i, D, log2_base, c, s);
+        rope_cs(pos, rf.inv[i], c, s);
         dst[i] = x1 * c - x2 * s;
         dst[i + D / 2] = x2 * c + x1 * s;
       }
@@ -113,11 +117,17 @@ decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int B, 
     const float lam = a.lambda[layer][h];
     float* S = a.state[layer] + ((long long)b * H + h) * D * D;
     const float vc = vv[col];
+    // all D/4 state loads of this thread are in flight before the first use
+    constexpr int RPT = D / 4;
+    float sv[RPT];
+#pragma unroll
+    for (int u = 0; u < RPT; ++u) sv[u] = S[(long long)(rg * RPT + u) * D + col];
     float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-    for (int r = rg * (D / 4); r < (rg + 1) * (D / 4); r += 2) {
-      const float s0 = lam * S[(long long)r * D + col] + kh[r] * vc;
-      const float s1 = lam * S[(long long)(r + 1) * D + col] + kh[r + 1] * vc;
+#pragma unroll
+    for (int u = 0; u < RPT; u += 2) {
+      const int r = rg * RPT + u;
+      const float s0 = lam * sv[u] + kh[r] * vc;
+      const float s1 = lam * sv[u + 1] + kh[r + 1] * vc;
       S[(long long)r * D + col] = s0;
       S[(long long)(r + 1) * D + col] = s1;
       acc0 = fmaf(qh[r], s0, acc0);
@@ -133,16 +143,17 @@ decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int B, 
     }
     return;
   }
-  // ---- sparse layer of batch b
-  const int b = blockIdx.x - n_lin;
-  const int G = Hq / Hkv;
+  // ---- sparse layer of batch b, rows [rc * 8, rc * 8 + 8) of its Hkv + Hq
+  const int b = (blockIdx.x - n_lin) / n_sp;
+  const int rc = (blockIdx.x - n_lin) % n_sp;
   const bool closes = ((pos + 1) % BLK) == 0;
-  float* qs = sh;                         // this CTA's q^ rows, reused per group
   const T* q = static_cast<const T*>(sp.q);
   const T* k = static_cast<const T*>(sp.k);
   const T* v = static_cast<const T*>(sp.v);
-  if (tid < 2 * Hkv) sp.counters[(long long)b * Hkv * 2 + tid] = 0u;
-  for (int r = warp; r < Hkv + Hq; r += 8) {
+  if (rc == 0 && tid < 2 * Hkv) sp.counters[(long long)b * Hkv * 2 + tid] = 0u;
+  {
+    const int r = rc * kDecodeRowsPerCta + warp;
+    if (warp >= kDecodeRowsPerCta || r >= Hkv + Hq) return;
     const bool isk = r < Hkv;
     const int h = isk ? r : r - Hkv;
     const T* src = isk ? k + ((long long)b * Hkv + h) * D : q + ((long long)b * Hq + h) * D;
@@ -173,21 +184,9 @@ decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int B, 
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < D / 32; ++e) {
-        sp.qhat[((long long)b * Hq + h) * D + lane + 32 * e] = x[e];
-        qsm[h * D + lane + 32 * e] = x[e];
-      }
+      for (int e = 0; e < D / 32; ++e) sp.qhat[((long long)b * Hq + h) * D + lane + 32 * e] = x[e];
     }
   }
-  __syncthreads();
-  // group sums (fixed order) from shared memory
-  for (int e = tid; e < Hkv * D; e += 256) {
-    const int g = e / D, d = e % D;
-    float s = 0.f;
-    for (int hh = 0; hh < G; ++hh) s += qsm[(g * G + hh) * D + d];
-    sp.qgrp[((long long)b * Hkv + g) * D + d] = s;
-  }
-  (void)qs;
 }
 
 // Top-k of the scored candidates: rows of the candidate chunks and, in the
@@ -198,9 +197,9 @@ decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int B, 
 // tie rule: equal scores go to the lower block).  Dynamic smem: chunk keys.
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads)
-decode_select_kernel(const float* __restrict__ qgrp, const float* __restrict__ kbar,
+decode_select_kernel(const float* __restrict__ qhat, const float* __restrict__ kbar,
                      uint32_t* __restrict__ cand_key, int32_t* __restrict__ cand_idx,
-                     int32_t* __restrict__ idx, unsigned* __restrict__ counters, int Hkv,
+                     int32_t* __restrict__ idx, unsigned* __restrict__ counters, int Hq, int Hkv,
                      long long cap_blocks, int bcur, int topk, int n_init, int n_local, int width,
                      int chunk, int n_chunks) {
   extern __shared__ uint32_t keys[];        // max(chunk, n_chunks * k) keys + as many ints
@@ -230,7 +229,13 @@ decode_select_kernel(const float* __restrict__ qgrp, const float* __restrict__ k
   }
   // ---- score this chunk
   const int c0 = ck * chunk, nc = min(chunk, n_cand - c0);
-  for (int e = tid; e < D; e += kSelectThreads) qv[e] = qgrp[((long long)b * Hkv + g) * D + e];
+  // group-summed query (fixed head order)
+  const int G = Hq / Hkv;
+  for (int e = tid; e < D; e += kSelectThreads) {
+    float s = 0.f;
+    for (int hh = 0; hh < G; ++hh) s += qhat[((long long)b * Hq + g * G + hh) * D + e];
+    qv[e] = s;
+  }
   __syncthreads();
   // one thread per candidate: its whole block-mean row is read with 16-byte
   // loads that are all independent, so many rows are in flight at once
@@ -298,176 +303,192 @@ decode_select_kernel(const float* __restrict__ qgrp, const float* __restrict__ k
   for (int e = n_first + k + n_loc + tid; e < width; e += kSelectThreads) row[e] = -1;
 }
 
-// Partial attention of the group's G heads over one selected block, then the
-// combine + gate in the last CTA of the (batch, kv head).  Keys / values are
-// staged as bf16 in shared memory with 16-byte chunks XOR-swizzled by row.
-// Partials: [B, Hkv, width, G, D + 4] = (m, l, -, -, o[D]) in base-2 logits.
+// Partial attention of the group's G heads over up to kDecodeBlocksPerCta
+// selected blocks (online softmax across them).  Keys / values are staged as
+// bf16 in shared memory with 16-byte chunks XOR-swizzled by row; the next
+// block's loads are in flight while the current one is processed.  Partials:
+// [B, Hkv, n_parts, G, D + 4] = (m, l, -, -, o[D]) in base-2 logits; they are
+// combined by decode_combine_kernel.
+constexpr int kDecodeBlocksPerCta = 1;
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 decode_attn_kernel(const float* __restrict__ qhat, const __nv_bfloat16* __restrict__ k_cache,
                    const __nv_bfloat16* __restrict__ v_cache, const int32_t* __restrict__ idx,
-                   float* __restrict__ part, unsigned* __restrict__ counters,
-                   const T* __restrict__ gate, T* __restrict__ out, int Hq, int Hkv,
-                   long long cap, long long pos, int BLK, int width, float sl2) {
+                   float* __restrict__ part, int Hq, int Hkv, long long cap, long long pos,
+                   int BLK, int width, int n_parts, float sl2) {
   constexpr int NC = D / 8;                 // 16-byte chunks per row
   constexpr int DP = D + 4;
+  constexpr int PER = 64 * NC / 256;        // 16-byte K (and V) chunks per thread and block
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint4* ks = reinterpret_cast<uint4*>(smem_raw);                 // [64][NC]
   uint4* vs = ks + 64 * NC;                                       // [64][NC]
   const int G = Hq / Hkv;
   float* qs = reinterpret_cast<float*>(vs + 64 * NC);             // [G][D]
   float* lg = qs + G * D;                                         // [G][64]
-  float* ml = lg + G * 64;                                        // [G][2]
-  __shared__ int s_last;
-  const int slot = blockIdx.x % width;
-  const int g = (blockIdx.x / width) % Hkv;
-  const int b = blockIdx.x / (width * Hkv);
+  float* os = lg + G * 64;                                        // [G][D] running outputs
+  float* ml = os + G * D;                                         // [G][2] running (m, l)
+  float* fs = ml + 2 * G;                                         // [G] rescale factors
+  const int pidx = blockIdx.x % n_parts;
+  const int g = (blockIdx.x / n_parts) % Hkv;
+  const int b = blockIdx.x / (n_parts * Hkv);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int j = idx[((long long)b * Hkv + g) * width + slot];
-  float* pbase = part + (((long long)b * Hkv + g) * width + slot) * G * DP;
-  const bool valid = j >= 0 && (long long)j * BLK <= pos;
-  if (j >= 0 && !valid) set_status(kStatusBounds);
-  if (!valid) {
-    // an empty slot: weight 0 in the combine, with finite (zero) partials
-    for (int e = tid; e < G * DP; e += 256) pbase[e] = (e % DP) == 0 ? -INFINITY : 0.f;
-  } else {
+  const int32_t* irow = idx + ((long long)b * Hkv + g) * width;
+  float* pbase = part + (((long long)b * Hkv + g) * n_parts + pidx) * G * DP;
+  const int slot0 = pidx * kDecodeBlocksPerCta;
+  const int nslot = min(kDecodeBlocksPerCta, width - slot0);
+  // blocks of this CTA that hold keys (entries of the list are ascending)
+  auto block_of = [&](int u) -> int {
+    const int j = irow[slot0 + u];
+    if (j >= 0 && (long long)j * BLK > pos) {
+      set_status(kStatusBounds);
+      return -1;
+    }
+    return j;
+  };
+  auto load_block = [&](int j, uint4* kr, uint4* vr) {
     const long long kend = ((long long)(j + 1) * BLK < pos + 1) ? (long long)(j + 1) * BLK : pos + 1;
     const int nk = (int)(kend - (long long)j * BLK);
-    // all loads of this thread are issued before the first shared-memory store
-    constexpr int PER = 64 * NC / 256;
-    uint4 kr[PER], vr[PER];
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
-      const int e = tid + 256 * u, s = e / NC, c = e % NC;
+      const int e = tid + 256 * u, sr = e / NC, c = e % NC;
       kr[u] = vr[u] = make_uint4(0, 0, 0, 0);
-      if (s < nk) {
-        const long long off = (((long long)b * cap + (long long)j * BLK + s) * Hkv + g) * D + 8 * c;
+      if (sr < nk) {
+        const long long off = (((long long)b * cap + (long long)j * BLK + sr) * Hkv + g) * D + 8 * c;
         kr[u] = *reinterpret_cast<const uint4*>(k_cache + off);
         vr[u] = *reinterpret_cast<const uint4*>(v_cache + off);
       }
     }
+    return nk;
+  };
+  {
     const float4* qsrc = reinterpret_cast<const float4*>(qhat + ((long long)b * Hq + g * G) * D);
     float4* qdst = reinterpret_cast<float4*>(qs);
     for (int e = tid; e < G * D / 4; e += 256) qdst[e] = qsrc[e];
+    for (int e = tid; e < G * D; e += 256) os[e] = 0.f;
+    for (int e = tid; e < G; e += 256) { ml[2 * e] = -INFINITY; ml[2 * e + 1] = 0.f; }
+  }
+  uint4 kr[PER], vr[PER];
+  int u = 0, j = -1, nk = 0;
+  while (u < nslot && (j = block_of(u)) < 0) ++u;
+  if (j >= 0) nk = load_block(j, kr, vr);
+  while (j >= 0) {
+    __syncthreads();                      // previous block's readers are done
 #pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int e = tid + 256 * u, s = e / NC, c = e % NC;
-      ks[s * NC + (c ^ (s & (NC - 1)))] = kr[u];
-      vs[s * NC + (c ^ (s & (NC - 1)))] = vr[u];
+    for (int w = 0; w < PER; ++w) {
+      const int e = tid + 256 * w, sr = e / NC, c = e % NC;
+      ks[sr * NC + (c ^ (sr & (NC - 1)))] = kr[w];
+      vs[sr * NC + (c ^ (sr & (NC - 1)))] = vr[w];
     }
+    const int cur_nk = nk;
+    // next block's loads overlap this block's arithmetic
+    int jn = -1;
+    ++u;
+    while (u < nslot && (jn = block_of(u)) < 0) ++u;
+    if (u >= nslot) jn = -1;
+    if (jn >= 0) nk = load_block(jn, kr, vr);
     __syncthreads();
     // logits: thread (key s, head hq + 4 m)
     {
-      const int s = tid & 63;
+      const int sr = tid & 63;
       for (int h = tid >> 6; h < G; h += 4) {
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         const float* qr = qs + h * D;
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
           float kf[8];
-          load8(reinterpret_cast<const __nv_bfloat16*>(&ks[s * NC + (c ^ (s & (NC - 1)))]), kf);
+          load8(reinterpret_cast<const __nv_bfloat16*>(&ks[sr * NC + (c ^ (sr & (NC - 1)))]), kf);
           a0 = fmaf(kf[0], qr[8 * c + 0], a0); a1 = fmaf(kf[1], qr[8 * c + 1], a1);
           a2 = fmaf(kf[2], qr[8 * c + 2], a2); a3 = fmaf(kf[3], qr[8 * c + 3], a3);
           a0 = fmaf(kf[4], qr[8 * c + 4], a0); a1 = fmaf(kf[5], qr[8 * c + 5], a1);
           a2 = fmaf(kf[6], qr[8 * c + 6], a2); a3 = fmaf(kf[7], qr[8 * c + 7], a3);
         }
-        lg[h * 64 + s] = s < nk ? ((a0 + a1) + (a2 + a3)) * sl2 : -INFINITY;
+        lg[h * 64 + sr] = sr < cur_nk ? ((a0 + a1) + (a2 + a3)) * sl2 : -INFINITY;
       }
     }
     __syncthreads();
-    // softmax per head (one warp per head, two logits per lane)
+    // online softmax per head (one warp per head, two logits per lane)
     for (int h = warp; h < G; h += 8) {
       const float x0 = lg[h * 64 + lane], x1 = lg[h * 64 + lane + 32];
-      const float m = warp_max(fmaxf(x0, x1));
-      const float p0 = exp2f(x0 - m), p1 = exp2f(x1 - m);
-      const float l = warp_sum(p0 + p1);
+      const float mo = ml[2 * h];
+      const float mn = fmaxf(mo, warp_max(fmaxf(x0, x1)));
+      const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn);
+      const float ls = warp_sum(p0 + p1);
       lg[h * 64 + lane] = p0;
       lg[h * 64 + lane + 32] = p1;
-      if (lane == 0) { ml[2 * h] = m; ml[2 * h + 1] = l; }
+      if (lane == 0) {
+        const float f = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+        fs[h] = f;
+        ml[2 * h] = mn;
+        ml[2 * h + 1] = ml[2 * h + 1] * f + ls;
+      }
     }
     __syncthreads();
-    // P V: thread (head, 8-column chunk)
+    // O = f O + P V: thread (head, 8-column chunk)
     for (int e = tid; e < G * NC; e += 256) {
       const int h = e / NC, c = e % NC;
-      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int s = 0; s < nk; ++s) {
+      float o[8];
+      const float f = fs[h];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) o[w] = os[h * D + 8 * c + w] * f;
+      for (int sr = 0; sr < cur_nk; ++sr) {
         float vf[8];
-        load8(reinterpret_cast<const __nv_bfloat16*>(&vs[s * NC + (c ^ (s & (NC - 1)))]), vf);
-        const float p = lg[h * 64 + s];
+        load8(reinterpret_cast<const __nv_bfloat16*>(&vs[sr * NC + (c ^ (sr & (NC - 1)))]), vf);
+        const float p = lg[h * 64 + sr];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) o[u] = fmaf(p, vf[u], o[u]);
+        for (int w = 0; w < 8; ++w) o[w] = fmaf(p, vf[w], o[w]);
       }
-      float* pr = pbase + h * DP;
-      *reinterpret_cast<float4*>(pr + 4 + 8 * c) = make_float4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<float4*>(pr + 8 + 8 * c) = make_float4(o[4], o[5], o[6], o[7]);
-      if (c == 0) { pr[0] = ml[2 * h]; pr[1] = ml[2 * h + 1]; }
+#pragma unroll
+      for (int w = 0; w < 8; ++w) os[h * D + 8 * c + w] = o[w];
     }
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0)
-    s_last = atomicAdd(counters + ((long long)b * Hkv + g) * 2 + 1, 1u) == (unsigned)(width - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // ---- combine the width partials of each head and apply the gate: the
-  // (m, l) pairs of every slot are staged in shared memory first, turned into
-  // weights 2^(m - M), then each thread streams its 8 output columns
-  const float* gb = part + ((long long)b * Hkv + g) * width * G * DP;
-  float* wgt = reinterpret_cast<float*>(smem_raw);        // [width][G] weights
-  float* lv = wgt + width * G;                            // [width][G] partial sums
-  float* lsum = lv + width * G;                           // [G]
-  for (int e = tid; e < width * G; e += 256) {
-    const float* pr = gb + (long long)e * DP;             // slot e / G, head e % G
-    wgt[e] = pr[0];
-    lv[e] = pr[1];
+    j = jn;
   }
   __syncthreads();
-  if (tid < G) {
+  // partial of this CTA (m = -inf, zeros when it held no key)
+  for (int e = tid; e < G * DP; e += 256) {
+    const int h = e / DP, c = e % DP;
+    pbase[e] = c == 0 ? ml[2 * h] : (c == 1 ? ml[2 * h + 1] : (c < 4 ? 0.f : os[h * D + c - 4]));
+  }
+}
+
+// Combine of the n_parts partials of one q head and the output gate: one CTA
+// per (batch, q head), one thread per output column.
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+decode_combine_kernel(const float* __restrict__ part, const T* __restrict__ gate,
+                      T* __restrict__ out, int Hq, int Hkv, int n_parts) {
+  constexpr int DP = D + 4;
+  extern __shared__ float wl[];                          // [n_parts] weights, [n_parts] sums
+  __shared__ float s_l;
+  const int hq = blockIdx.x % Hq;
+  const int b = blockIdx.x / Hq;
+  const int G = Hq / Hkv, g = hq / G, h = hq % G;
+  const int tid = threadIdx.x;
+  const float* pb = part + (((long long)b * Hkv + g) * n_parts * G + h) * DP;
+  const long long pstride = (long long)G * DP;
+  for (int e = tid; e < n_parts; e += D) {
+    wl[e] = pb[e * pstride];
+    wl[n_parts + e] = pb[e * pstride + 1];
+  }
+  __syncthreads();
+  if (tid < 32) {
     float M = -INFINITY;
-    for (int sl = 0; sl < width; ++sl) M = fmaxf(M, wgt[sl * G + tid]);
+    for (int e = tid; e < n_parts; e += 32) M = fmaxf(M, wl[e]);
+    M = warp_max(M);
     float L = 0.f;
-    for (int sl = 0; sl < width; ++sl) {
-      const float m = wgt[sl * G + tid];
-      const float f = m == -INFINITY ? 0.f : exp2f(m - M);
-      wgt[sl * G + tid] = f;
-      L = fmaf(f, lv[sl * G + tid], L);
+    for (int e = tid; e < n_parts; e += 32) {
+      const float f = wl[e] == -INFINITY ? 0.f : exp2f(wl[e] - M);
+      L = fmaf(f, wl[n_parts + e], L);
+      wl[e] = f;
     }
-    lsum[tid] = L;
+    L = warp_sum(L);
+    if (tid == 0) s_l = L;
   }
   __syncthreads();
-  for (int e = tid; e < G * NC; e += 256) {
-    const int h = e / NC, c = e % NC;
-    const float L = lsum[h];
-    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    // 8 slots per batch: their 16 loads are issued before any is used
-    for (int s0 = 0; s0 < width; s0 += 8) {
-      float4 a[8], bq[8];
-      float f[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int sl = min(s0 + u, width - 1);
-        const float* pr = gb + ((long long)sl * G + h) * DP;
-        a[u] = *reinterpret_cast<const float4*>(pr + 4 + 8 * c);
-        bq[u] = *reinterpret_cast<const float4*>(pr + 8 + 8 * c);
-        f[u] = s0 + u < width ? wgt[sl * G + h] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        o[0] = fmaf(f[u], a[u].x, o[0]); o[1] = fmaf(f[u], a[u].y, o[1]);
-        o[2] = fmaf(f[u], a[u].z, o[2]); o[3] = fmaf(f[u], a[u].w, o[3]);
-        o[4] = fmaf(f[u], bq[u].x, o[4]); o[5] = fmaf(f[u], bq[u].y, o[5]);
-        o[6] = fmaf(f[u], bq[u].z, o[6]); o[7] = fmaf(f[u], bq[u].w, o[7]);
-      }
-    }
-    const long long off = ((long long)b * Hq + g * G + h) * D + 8 * c;
-    float gv[8];
-    load8(gate + off, gv);
-    const float inv = 1.f / L;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) gv[u] = sigmoidf_(gv[u]) * o[u] * inv;
-    store8(out + off, gv);
-  }
+  float o = 0.f;
+  for (int e = 0; e < n_parts; ++e) o = fmaf(wl[e], pb[e * pstride + 4 + tid], o);
+  const long long off = ((long long)b * Hq + hq) * D + tid;
+  out[off] = from_f32<T>(sigmoidf_(to_f32(gate[off])) * o / s_l);
 }
 
 }  // namespace sala

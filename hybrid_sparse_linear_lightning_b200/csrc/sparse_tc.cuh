@@ -9,10 +9,12 @@
 // once for all 256 query rows (GQA sharing without multicast).
 //
 // Per selected block j (64 keys):  S_t = Q_t K_j^T  (tcgen05, M=128 N=64,
-// fp32 in TMEM);  softmax warps read S_t one row per thread, apply the causal
-// mask on the diagonal block, exponentiate against a running max, write
-// P_t (bf16 pairs) back to TMEM;  O_t += P_t V_j  (tcgen05 with A read from
-// TMEM, M=128 N=d, fp32 in TMEM).  Exact softmax: the running max is raised (and O, l rescaled) only
+// fp32 in TMEM, two buffers per tile);  softmax warps read S_t one row per
+// thread, apply the causal mask on the diagonal block, exponentiate against a
+// running max and write P_t (bf16 pairs) over the S_t buffer they read;
+// O_t += P_t V_j  (tcgen05 with A read from TMEM, M=128 N=d, fp32 in TMEM).
+// S_t of block j+1 is issued before P_t V_j, into the other buffer, so the
+// softmax of block j+1 starts as soon as P_t of block j is written.  Exact softmax: the running max is raised (and O, l rescaled) only
 // when a row's max grows by more than 2^8, so values stay bounded; the final
 // division by l makes the result independent of that choice up to rounding.
 // Epilogue: out = sigmoid(gate) * O / l.
@@ -33,6 +35,7 @@ constexpr int kSpTcThreads = 384;
 constexpr int kSpTcStages = 4;
 constexpr int kSpTcHeadsPerCta = 4;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kSpPolyPairsPer8 = 2;         // exponential pairs evaluated on the FMA pipe
 
 template <int D>
 struct SpTcLayout {
@@ -42,15 +45,16 @@ struct SpTcLayout {
   static constexpr int kQ = 0;
   static constexpr int kKVBase = kQ + 2 * kQTile;
   static constexpr int kBar = kKVBase + kSpTcStages * 2 * kKV;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], o_done[2], fin
-  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 8 + 1;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_full[2], o_done[2], fin
+  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 4 + 4 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kSel = kMisc + 16;               // int sel[width]
   static constexpr int kBytes(int width) { return kSel + 4 * width; }
   static constexpr int kTmemCols = 512;
-  // TMEM columns: S_0, S_1 (64 fp32 each), O_0, O_1 (D each), P_0, P_1 (64 bf16 = 32 each)
-  static constexpr int kColS0 = 0, kColS1 = 64, kColO0 = 128, kColO1 = 128 + D;
-  static constexpr int kColP0 = 128 + 2 * D, kColP1 = kColP0 + 32;
+  // TMEM columns: S of tile t, buffer x at 64 (2 t + x) (64 fp32; P of the
+  // same block overwrites its first 32 columns as bf16 pairs), O_0, O_1 (D each)
+  static constexpr int col_s(int t, int x) { return 64 * (2 * t + x); }
+  static constexpr int kColO0 = 256, kColO1 = 256 + D;
 };
 
 template <typename T, int D>
@@ -68,9 +72,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kSpTcStages;
-  uint64_t* s_full = kv_empty + kSpTcStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
+  uint64_t* s_full = kv_empty + kSpTcStages;   // [tile * 2 + buffer]
+  uint64_t* p_full = s_full + 4;
   uint64_t* o_done = p_full + 2;
   uint64_t* fin = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -95,8 +98,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::mbar_init(kv_empty + s, 1);
     }
     for (int t = 0; t < 2; ++t) {
-      tc::mbar_init(s_full + t, 1);
-      tc::mbar_init(s_free + t, 4);
+      tc::mbar_init(s_full + 2 * t, 1);
+      tc::mbar_init(s_full + 2 * t + 1, 1);
       tc::mbar_init(p_full + t, 4);
       tc::mbar_init(o_done + t, 1);
     }
@@ -159,8 +162,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = tc::smem_u32(sQ), kv_addr = tc::smem_u32(sKV);
-      // Issue order: S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...  so the
-      // softmax of one tile overlaps the tensor work of the other.
+      // Issue order: S_0(0) S_1(0) | S_0(j+1) S_1(j+1) PV_0(j) PV_1(j) | ...  S of
+      // the next block goes into the other buffer of its tile (free once
+      // P V of block j-1 has completed), so it is ready when the softmax of
+      // block j finishes.
       auto issue_s = [&](int t, int j) {
         const uint32_t k_addr = kv_addr + (j % kSpTcStages) * 2 * L::kKV;
 #pragma unroll
@@ -168,16 +173,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
           const uint32_t off = (kk & 3) * 32;   // 16 elements = 32 B inside the atom
           const uint64_t ad = tc::smem_desc_sw128(q_addr + t * L::kQTile + (kk >> 2) * (128 * 128) + off, 16, 1024);
           const uint64_t bd = tc::smem_desc_sw128(k_addr + (kk >> 2) * (64 * 128) + off, 16, 1024);
-          tc::mma_bf16_ss(tmem + (t ? L::kColS1 : L::kColS0), ad, bd, idesc_s, kk > 0);
+          tc::mma_bf16_ss(tmem + L::col_s(t, j & 1), ad, bd, idesc_s, kk > 0);
         }
-        tc::mma_commit(s_full + t);
+        tc::mma_commit(s_full + 2 * t + (j & 1));
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t v_addr = kv_addr + (j % kSpTcStages) * 2 * L::kKV + L::kKV;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = tc::smem_desc_sw128(v_addr + kk * 2048, 64 * 128, 1024);
-          tc::mma_bf16_ts(tmem + (t ? L::kColO1 : L::kColO0), tmem + (t ? L::kColP1 : L::kColP0) + kk * 8,
+          tc::mma_bf16_ts(tmem + (t ? L::kColO1 : L::kColO0), tmem + L::col_s(t, j & 1) + kk * 8,
                           bd, idesc_o, (j > 0 || kk > 0));
         }
         tc::mma_commit(o_done + t);
@@ -189,19 +194,22 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         issue_s(1, 0);
       }
       for (int j = 0; ok && j < n_sel; ++j) {
-        const bool more = j + 1 < n_sel;
+        if (j + 1 < n_sel) {
+          if (!(ok = tc::mbar_wait(kv_full + (j + 1) % kSpTcStages, ((j + 1) / kSpTcStages) & 1))) break;
+          for (int t = 0; t < 2 && ok; ++t) {
+            // buffer (j+1) & 1 last held P of block j-1
+            if (j >= 1 && !(ok = tc::mbar_wait(o_done + t, (j - 1) & 1))) break;
+            tc::tc_fence_after();
+            issue_s(t, j + 1);
+          }
+          if (!ok) break;
+        }
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = tc::mbar_wait(p_full + t, j & 1))) break;
           tc::tc_fence_after();
           issue_pv(t, j);
-          if (t == 1) tc::mma_commit(kv_empty + (j % kSpTcStages));
-          if (more) {
-            if (t == 0 && !(ok = tc::mbar_wait(kv_full + (j + 1) % kSpTcStages, ((j + 1) / kSpTcStages) & 1))) break;
-            if (!(ok = tc::mbar_wait(s_free + t, j & 1))) break;
-            tc::tc_fence_after();
-            issue_s(t, j + 1);
-          }
         }
+        if (ok) tc::mma_commit(kv_empty + (j % kSpTcStages));
       }
       // drain: every MMA issued above has completed once `fin` fires
       tc::mma_commit(fin);
@@ -214,23 +222,19 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     const int r = quad * 32 + lane;           // row in the tile
     const int tok = r & 63;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t s_addr = lane_base + (t ? L::kColS1 : L::kColS0);
     const uint32_t o_addr = lane_base + (t ? L::kColO1 : L::kColO0);
-    const uint32_t p_addr = lane_base + (t ? L::kColP1 : L::kColP0);
     const float2 sl2v = make_float2(sl2, sl2);
     float m = -INFINITY, l = 0.f;
     bool ok = n_sel > 0;
     for (int j = 0; ok && j < n_sel; ++j) {
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(s_full + t, j & 1));
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(s_full + 2 * t + (j & 1), (j >> 1) & 1));
       if (!ok) break;
       tc::tc_fence_after();
+      const uint32_t s_addr = lane_base + L::col_s(t, j & 1);   // P of block j goes here too
       float x[64];
       tc::tmem_ld32(s_addr, x);
       tc::tmem_ld32(s_addr + 32, x + 32);
       tc::tmem_wait_ld();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(s_free + t);
       // causal mask on the diagonal block only (warp-uniform branch)
       if (sel[j] == i) {
 #pragma unroll
@@ -246,9 +250,11 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * sl2;
       if (j == 0) m = mx;
       if (j > 0) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
-        if (!ok) break;
+        // O is rescaled (after P V of block j-1 has landed) only when a row's
+        // max grew by more than the threshold
         if (__any_sync(0xffffffffu, mx > m + kRescaleThreshold)) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
+          if (!ok) break;
           const float mnew = fmaxf(m, mx);
           const float f = exp2f(m - mnew);
           m = mnew;
@@ -274,14 +280,24 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float2 tt = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sl2v, negm);
-        const float2 pv = make_float2(tc::ex2_approx(tt.x), tc::ex2_approx(tt.y));
+        // kSpPolyPairsPer8 of every 8 pairs on the FMA pipe, the rest on the
+        // special-function unit
+        const float2 pv = (e & 7) < kSpPolyPairsPer8
+                              ? tc::exp2_fma2(tt)
+                              : make_float2(tc::ex2_approx(tt.x), tc::ex2_approx(tt.y));
         acc4[e & 3] = __fadd2_rn(acc4[e & 3], pv);
         __nv_bfloat162 h2 = __floats2bfloat162_rn(pv.x, pv.y);
         pk[e] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      tc::tmem_st32_u(p_addr, pk);
+      tc::tmem_st32_u(s_addr, pk);
       const float2 s01 = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
       l += s01.x + s01.y;
+      // P V of block j-1 has completed before P of block j is published, so
+      // o_done never runs more than one phase ahead of a parity wait on it
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
+        if (!ok) break;
+      }
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
