@@ -485,8 +485,15 @@ decode_combine_kernel(const float* __restrict__ part, const T* __restrict__ gate
     if (tid == 0) s_l = L;
   }
   __syncthreads();
-  float o = 0.f;
-  for (int e = 0; e < n_parts; ++e) o = fmaf(wl[e], pb[e * pstride + 4 + tid], o);
+  // 8 independent partial sums so that the loads of 8 partials overlap
+  float o8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int e = 0;
+  for (; e + 8 <= n_parts; e += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o8[u] = fmaf(wl[e + u], pb[(e + u) * pstride + 4 + tid], o8[u]);
+  }
+  for (; e < n_parts; ++e) o8[0] = fmaf(wl[e], pb[e * pstride + 4 + tid], o8[0]);
+  const float o = ((o8[0] + o8[1]) + (o8[2] + o8[3])) + ((o8[4] + o8[5]) + (o8[6] + o8[7]));
   const long long off = ((long long)b * Hq + hq) * D + tid;
   out[off] = from_f32<T>(sigmoidf_(to_f32(gate[off])) * o / s_l);
 }
