@@ -75,6 +75,19 @@ inline float sparse_scale(const sala_sparse_desc* d) {
   return d->scale > 0.f ? d->scale : 1.0f / sqrtf((float)d->head_dim);
 }
 
+// Failure-detection self-test: one thread waits, with the library's bounded
+// wait, on an mbarrier that no thread arrives at.  The wait runs out, sets
+// the timeout bit of the status word and the kernel returns.
+__global__ void selftest_unarrived_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)tc::mbar_wait(&bar, 0);
+}
+
 struct LinearWs {
   size_t qn, kn, seg, total;
 };
@@ -583,6 +596,13 @@ sala_status sala_get_device_status(void* stream) {
   if (v & kStatusTimeout) return SALA_ERR_TIMEOUT;
   if (v & kStatusBounds) return SALA_ERR_DEVICE_FAULT;
   return SALA_OK;
+}
+
+sala_status sala_selftest_bounded_wait(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  selftest_unarrived_wait_kernel<<<1, 32, 0, st>>>();
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  return sala_get_device_status(stream);
 }
 
 int sala_version(void) { return 100; }

@@ -33,7 +33,7 @@ EXPORTED = [
     "sala_sparse_workspace_size", "sala_sparse_select", "sala_sparse_prefill",
     "sala_decode_workspace_size", "sala_decode_step", "sala_status_string",
     "sala_get_device_status", "sala_version", "sala_kernel_launch_count",
-    "sala_sparse_select_noalloc",
+    "sala_sparse_select_noalloc", "sala_selftest_bounded_wait",
 ]
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -93,6 +93,7 @@ def _load():
         "sala_version": (I, []),
         "sala_kernel_launch_count": (ctypes.c_uint64, []),
         "sala_sparse_select_noalloc": (I, [P] + [P] * 8 + [P]),
+        "sala_selftest_bounded_wait": (I, [P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -211,6 +212,10 @@ def sala_decode_step(d: DecodeDesc, io: DecodeIO, k_cache, v_cache, kbar, ksum, 
 
 def sala_get_device_status(stream=None) -> int:
     return int(LIB.sala_get_device_status(_stream(stream)))
+
+
+def sala_selftest_bounded_wait(stream=None) -> int:
+    return int(LIB.sala_selftest_bounded_wait(_stream(stream)))
 
 
 def sala_version() -> int:

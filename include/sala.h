@@ -204,6 +204,16 @@ const char* sala_status_string(sala_status s);
  * word: SALA_OK, SALA_ERR_TIMEOUT or SALA_ERR_DEVICE_FAULT. */
 sala_status sala_get_device_status(void* stream);
 
+/* Failure-detection self-test (no counterpart on the pages; test support).
+ * Launches one single-CTA kernel on `stream` that waits on an mbarrier no
+ * thread ever arrives at.  The wait is bounded like every wait in the
+ * library (about 2^31 SM cycles, roughly a second); when it runs out the
+ * kernel sets the timeout bit of the status word and returns, leaving the
+ * context usable.  Returns what sala_get_device_status() then reports
+ * (SALA_ERR_TIMEOUT when the bound works) and clears the word, or
+ * SALA_ERR_CUDA if the launch fails. */
+sala_status sala_selftest_bounded_wait(void* stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int sala_version(void);
 
