@@ -88,6 +88,15 @@ __global__ void selftest_unarrived_wait_kernel() {
   if (threadIdx.x == 0) (void)tc::mbar_wait(&bar, 0);
 }
 
+// base^(-2i/D) for i < D/2 in fp64
+RopeFreq rope_freq(int D, float base) {
+  RopeFreq rf;
+  memset(&rf, 0, sizeof(rf));
+  const double log2_base = log2((double)base);
+  for (int i = 0; i < D / 2; ++i) rf.inv[i] = exp2(-2.0 * i / D * log2_base);
+  return rf;
+}
+
 struct LinearWs {
   size_t qn, kn, seg, total;
 };
@@ -125,7 +134,7 @@ sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, 
   const int pro_blocks = (int)((tokens + kRopeTokens - 1) / kRopeTokens);
   linear_prologue_kernel<T, D><<<pro_blocks, kPrologueThreads, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), wq, wk, qn, kn, tokens, d->seqlen,
-      d->heads, d->pos0, log2((double)d->rope_base), d->rms_eps);
+      d->heads, d->pos0, rope_freq(D, d->rope_base), d->rms_eps);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
   // bf16 activations with head_dim 128 run on the tensor cores; fp32
   // activations and head_dim 64 on CUDA cores.
@@ -348,10 +357,7 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   sp.qhat = reinterpret_cast<float*>(ws + w.qhat);
   sp.counters = reinterpret_cast<unsigned*>(ws + w.counters);
   // 1. linear layers + sparse prep
-  RopeFreq rf;
-  memset(&rf, 0, sizeof(rf));
-  const double log2_base = log2((double)L.rope_base);
-  for (int i = 0; i < D / 2; ++i) rf.inv[i] = exp2(-2.0 * i / D * log2_base);
+  const RopeFreq rf = rope_freq(D, L.rope_base);
   const int n_lin = d->n_linear * L.batch * L.heads * (D / 64);
   const int n_sp = (S.kv_heads + S.q_heads + kDecodeRowsPerCta - 1) / kDecodeRowsPerCta;
   decode_stage1_kernel<T, D><<<n_lin + S.batch * n_sp, 256, 0, st>>>(

@@ -50,10 +50,6 @@ struct DecodeSparseArgs {
   unsigned* counters;   // [B, Hkv, 2]: selection completion counts (second unused)
 };
 
-// RoPE inverse frequencies base^(-2i/D), i < D/2, formed in fp64 on the host.
-struct RopeFreq {
-  double inv[64];
-};
 
 // cos / sin of p * base^(-2i/D): the argument is formed and reduced modulo
 // 2 pi in fp64 (|p| < 2^53), then evaluated in fp32 on [-pi, pi].

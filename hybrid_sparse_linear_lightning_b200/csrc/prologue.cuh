@@ -12,6 +12,11 @@
 namespace sala {
 
 constexpr int kPrologueThreads = 256;
+
+// RoPE inverse frequencies base^(-2i/D), i < D/2, formed in fp64 on the host.
+struct RopeFreq {
+  double inv[64];
+};
 constexpr int kRopeTokens = 4;   // tokens per CTA of the linear prologue
 
 // Thread layout: a "row" is one (token, head) vector of D elements, handled by
@@ -51,19 +56,18 @@ __device__ __forceinline__ void rope_pair8(float* lo, float* hi, const float* c,
 }
 
 // cos / sin of (pos0 + t) * theta_i for `ntok` tokens starting at token t0 of
-// a sequence of length N (flattened index over batch * N), computed in fp64
-// with the argument formed exactly in fp64 and rounded to fp32 afterwards.
+// a sequence of length N (flattened index over batch * N): the argument is
+// formed and reduced modulo 2 pi in fp64 (|p| < 2^53), then evaluated in fp32
+// on [-pi, pi].
 template <int D>
 __device__ __forceinline__ void rope_table(float* cs, float* sn, long long tok0, int ntok,
-                                           int N, long long pos0, double log2_base) {
+                                           int N, long long pos0, const RopeFreq& rf) {
   for (int e = threadIdx.x; e < ntok * (D / 2); e += blockDim.x) {
     const int tt = e / (D / 2), i = e % (D / 2);
     const long long p = pos0 + (tok0 + tt) % N;
-    const double theta = exp2(-2.0 * i / D * log2_base);
-    double sv, cv;
-    sincos((double)p * theta, &sv, &cv);
-    cs[e] = (float)cv;
-    sn[e] = (float)sv;
+    const double a = (double)p * rf.inv[i];
+    const double two_pi = 6.283185307179586476925286766559;
+    sincosf((float)(a - rint(a / two_pi) * two_pi), &sn[e], &cs[e]);
   }
 }
 
@@ -75,13 +79,13 @@ linear_prologue_kernel(const T* __restrict__ q, const T* __restrict__ k,
                        const float* __restrict__ wq, const float* __restrict__ wk,
                        __nv_bfloat16* __restrict__ qn, __nv_bfloat16* __restrict__ kn,
                        long long total_tokens, int N, int H, long long pos0,
-                       double log2_base, float eps) {
+                       const RopeFreq rf, float eps) {
   constexpr int TPR = D / 16;
   __shared__ float cs[kRopeTokens * D / 2];
   __shared__ float sn[kRopeTokens * D / 2];
   const long long tok0 = (long long)blockIdx.x * kRopeTokens;
   const int ntok = (int)(total_tokens - tok0 < kRopeTokens ? total_tokens - tok0 : kRopeTokens);
-  rope_table<D>(cs, sn, tok0, ntok, N, pos0, log2_base);
+  rope_table<D>(cs, sn, tok0, ntok, N, pos0, rf);
   __syncthreads();
 
   const int c = threadIdx.x % TPR;
