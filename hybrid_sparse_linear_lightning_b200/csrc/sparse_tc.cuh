@@ -45,8 +45,9 @@ struct SpTcLayout {
   static constexpr int kQ = 0;
   static constexpr int kKVBase = kQ + 2 * kQTile;
   static constexpr int kBar = kKVBase + kSpTcStages * 2 * kKV;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_full[2], o_done[2], fin
-  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 4 + 4 + 1;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_full[2],
+  // o_done[tile][block parity], fin
+  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 4 + 2 + 4 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kSel = kMisc + 16;               // int sel[width]
   static constexpr int kBytes(int width) { return kSel + 4 * width; }
@@ -74,8 +75,12 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* kv_empty = kv_full + kSpTcStages;
   uint64_t* s_full = kv_empty + kSpTcStages;   // [tile * 2 + buffer]
   uint64_t* p_full = s_full + 4;
+  // P V of block j of tile t completes o_done[2 t + (j & 1)]: every wait on it
+  // (for block j-1, by the MMA issuer before S of block j+1, by the softmax
+  // before a rescale and before the epilogue) comes after P V of block j-3
+  // has completed, so a parity wait is never more than one phase behind
   uint64_t* o_done = p_full + 2;
-  uint64_t* fin = o_done + 2;
+  uint64_t* fin = o_done + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   int* n_sel_slot = reinterpret_cast<int*>(smem + L::kMisc + 4);
   int* sel = reinterpret_cast<int*>(smem + L::kSel);
@@ -101,7 +106,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::mbar_init(s_full + 2 * t, 1);
       tc::mbar_init(s_full + 2 * t + 1, 1);
       tc::mbar_init(p_full + t, 4);
-      tc::mbar_init(o_done + t, 1);
+      tc::mbar_init(o_done + 2 * t, 1);
+      tc::mbar_init(o_done + 2 * t + 1, 1);
     }
     tc::mbar_init(fin, 1);
     tc::fence_barrier_init();
@@ -185,7 +191,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
           tc::mma_bf16_ts(tmem + (t ? L::kColO1 : L::kColO0), tmem + L::col_s(t, j & 1) + kk * 8,
                           bd, idesc_o, (j > 0 || kk > 0));
         }
-        tc::mma_commit(o_done + t);
+        tc::mma_commit(o_done + 2 * t + (j & 1));
       };
       bool ok = tc::mbar_wait(q_full, 0) && tc::mbar_wait(kv_full, 0);
       if (ok) {
@@ -198,7 +204,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
           if (!(ok = tc::mbar_wait(kv_full + (j + 1) % kSpTcStages, ((j + 1) / kSpTcStages) & 1))) break;
           for (int t = 0; t < 2 && ok; ++t) {
             // buffer (j+1) & 1 last held P of block j-1
-            if (j >= 1 && !(ok = tc::mbar_wait(o_done + t, (j - 1) & 1))) break;
+            if (j >= 1 && !(ok = tc::mbar_wait(o_done + 2 * t + ((j - 1) & 1), ((j - 1) >> 1) & 1))) break;
             tc::tc_fence_after();
             issue_s(t, j + 1);
           }
@@ -253,7 +259,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         // O is rescaled (after P V of block j-1 has landed) only when a row's
         // max grew by more than the threshold
         if (__any_sync(0xffffffffu, mx > m + kRescaleThreshold)) {
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
+          ok = __all_sync(0xffffffffu,
+                          tc::mbar_wait(o_done + 2 * t + ((j - 1) & 1), ((j - 1) >> 1) & 1));
           if (!ok) break;
           const float mnew = fmaxf(m, mx);
           const float f = exp2f(m - mnew);
@@ -292,19 +299,15 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::tmem_st32_u(s_addr, pk);
       const float2 s01 = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
       l += s01.x + s01.y;
-      // P V of block j-1 has completed before P of block j is published, so
-      // o_done never runs more than one phase ahead of a parity wait on it
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (j - 1) & 1));
-        if (!ok) break;
-      }
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(p_full + t);
     }
     // epilogue: out = sigmoid(gate) * O / l
-    if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(o_done + t, (n_sel - 1) & 1));
+    if (ok)
+      ok = __all_sync(0xffffffffu,
+                      tc::mbar_wait(o_done + 2 * t + ((n_sel - 1) & 1), ((n_sel - 1) >> 1) & 1));
     if (ok) {
       tc::tc_fence_after();
       const int head = hbase + 2 * t + (r >> 6);
