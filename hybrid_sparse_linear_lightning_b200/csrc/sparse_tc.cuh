@@ -6,7 +6,7 @@
 // 64 tokens of every q head of the group share one list of selected key
 // blocks, so a CTA takes FOUR q heads of the group (two 128-row tiles: 2 heads
 // x 64 tokens each) and streams each selected K/V block through shared memory
-// once for all 256 query rows (GQA sharing without multicast).
+// once for all 256 query rows (GQA sharing: one K/V fetch per CTA).
 //
 // Per selected block j (64 keys):  S_t = Q_t K_j^T  (tcgen05, M=128 N=64,
 // fp32 in TMEM, two buffers per tile);  softmax warps read S_t one row per
