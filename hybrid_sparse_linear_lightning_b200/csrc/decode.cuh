@@ -66,7 +66,7 @@ __device__ __forceinline__ void rope_cs(long long p, double inv_freq, float& c, 
 // Hkv keys and Hq queries of batch b (normalise k and append it and v to the
 // caches, update the running block sum / mean; normalise q); the first of
 // them also resets the completion counters.
-constexpr int kDecodeMaxQHeads = 64;   // q heads of the sparse layer (selection staging)
+constexpr int kDecodeMaxQHeads = 64;   // largest sparse-layer q head count the decode step takes
 constexpr int kDecodeRowsPerCta = 8;   // sparse-layer rows per stage-1 CTA
 
 template <typename T, int D>
