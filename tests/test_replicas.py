@@ -58,3 +58,19 @@ def test_reference_arm_rank_nonzero_exits_silently():
                        text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_line_rank0(capsys):
+    """The oracle arm on rank 0: one JSON line whose step time is the
+    extrapolated time of a whole step at its own throughput."""
+    import json
+    import types
+    import bench
+    os.environ.pop("RANK", None)
+    bench.run_reference(types.SimpleNamespace(workload="group_256k", steps=1, warmup=0))
+    line = capsys.readouterr().out.strip().splitlines()[-1]
+    d = json.loads(line)
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    tokens = 262144
+    assert d["ms_per_step"] == pytest.approx(tokens / d["value"] * 1e3, rel=1e-3)
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
