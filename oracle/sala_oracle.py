@@ -39,9 +39,17 @@ its function) are the plainest ones consistent with the pages:
 * Exact softmax attention (scale 1/sqrt(d)) of each query over the keys of
   its selected blocks at positions <= its own.
 
-All arithmetic is fp64 except the block-selection decision, which (a float
-comparison deciding an integer result) is taken in fp32, the precision of the
-CUDA kernels, unless ``score_dtype=np.float64`` is passed.
+All arithmetic is fp64, the block-selection decision included: the selected
+index sets are exact for the fp64 scores, and an implementation that ranks
+in lower precision may differ from them only where the k-th and (k+1)-th
+candidate scores lie within a relative 1e-3 of each other (the tolerance
+stated for the selected indices).  ``score_dtype`` can still be lowered for
+experiments; nothing on the test path does so.
+
+Full-size inputs (up to 1M tokens, 32 query heads) do not fit in host memory
+as fp64 arrays, so the sparse layer also has ``*_rows`` forms that take the
+queries of a chosen subset of query blocks only; they compute the same
+definitions for those blocks (pinned against the full forms).
 """
 from __future__ import annotations
 
@@ -55,6 +63,7 @@ __all__ = [
     "linear_attention_quadratic", "linear_layer",
     "block_means", "block_scores", "select_row", "select_blocks",
     "selected_count", "sparse_attention", "sparse_select", "sparse_layer",
+    "sparse_attention_rows", "sparse_select_rows", "sparse_layer_rows",
     "decode_linear_step", "decode_sparse_step",
 ]
 
@@ -235,21 +244,23 @@ def block_means(x, block, dtype=F64):
     return np.ascontiguousarray(np.transpose(m, (0, 2, 1, 3)))
 
 
-def block_scores(qbar, kbar, dtype=F64):
+def block_scores(qbar, kbar, dtype=F64, rows=None):
     """Block scores s[b, g, i, j] = <sum_{h in G(g)} qbar_i^h, kbar_j^g> / sqrt(d).
 
-    qbar: [B, Hq, nb, d] per-head query block means; kbar: [B, Hkv, nb, d].
+    qbar: [B, Hq, nq, d] per-head query block means; kbar: [B, Hkv, nb, d].
     Query heads h with h // (Hq/Hkv) == g form the group G(g) (GQA).
-    Entries with j > i (non-causal) are -inf.
+    Entries with j > i (non-causal) are -inf.  Query block r of qbar is
+    block ``rows[r]`` of the sequence (default: block r, nq == nb).
     """
     qbar = np.asarray(qbar, dtype)
     kbar = np.asarray(kbar, dtype)
-    B, Hq, nb, d = qbar.shape
-    Hkv = kbar.shape[1]
+    B, Hq, nq, d = qbar.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
     G = Hq // Hkv
-    qg = qbar.reshape(B, Hkv, G, nb, d).sum(axis=2, dtype=dtype)
+    qg = qbar.reshape(B, Hkv, G, nq, d).sum(axis=2, dtype=dtype)
     s = np.einsum("bgid,bgjd->bgij", qg, kbar) / dtype(math.sqrt(d))
-    causal = np.tril(np.ones((nb, nb), dtype=bool))
+    qi = np.arange(nq) if rows is None else np.asarray(rows)
+    causal = np.arange(nb)[None, :] <= qi[:, None]
     return np.where(causal[None, None], s, -np.inf)
 
 
@@ -299,22 +310,55 @@ def select_blocks(scores, topk, n_init, n_local, rows=None):
     return idx
 
 
+def _selection_inputs(x, w, eps, block, sd, exact):
+    """Block means of the normalised rows of x in the precision ``sd`` of the
+    ranking (the fp64 normalised values themselves when sd is fp64)."""
+    xs = exact if sd is F64 else rms_norm(np.asarray(x, sd), np.asarray(w, sd), eps, dtype=sd)
+    return block_means(xs, block, sd)
+
+
 def sparse_select(q, k, wq, wk, *, block=64, topk=16, n_init=1, n_local=2, eps=1e-6,
-                  score_dtype=np.float32, rows=None):
+                  score_dtype=F64, rows=None):
     """Selection stage of the sparse layer (NoPE: no RoPE in sparse layers).
 
-    Returns (q_hat, k_hat, kbar, idx, scores) with q_hat/k_hat/kbar in fp64
-    and scores / idx computed with ``score_dtype`` arithmetic throughout
-    (normalisation, block means, group sum, dot product).
+    Returns (q_hat, k_hat, kbar, idx, scores): q_hat / k_hat / kbar in fp64,
+    scores [B, Hkv, nb, nb] and idx [B, Hkv, nb, W] ranked in ``score_dtype``
+    (fp64 by default) throughout (normalisation, block means, group sum, dot
+    product).  ``rows`` restricts the index lists to those query blocks.
     """
     qh = rms_norm(q, wq, eps)
     kh = rms_norm(k, wk, eps)
     kbar = block_means(kh, block)
     sd = score_dtype
-    q_s = rms_norm(np.asarray(q, sd), np.asarray(wq, sd), eps, dtype=sd)
-    k_s = rms_norm(np.asarray(k, sd), np.asarray(wk, sd), eps, dtype=sd)
-    scores = block_scores(block_means(q_s, block, sd), block_means(k_s, block, sd), sd)
+    scores = block_scores(_selection_inputs(q, wq, eps, block, sd, qh),
+                          _selection_inputs(k, wk, eps, block, sd, kh), sd)
     idx = select_blocks(scores, topk, n_init, n_local, rows)
+    return qh, kh, kbar, idx, scores
+
+
+def sparse_select_rows(q_rows, rows, k, wq, wk, *, block=64, topk=16, n_init=1, n_local=2,
+                       eps=1e-6, score_dtype=F64):
+    """Selection of the query blocks ``rows`` only.
+
+    q_rows: [B, R*block, Hq, d], the raw queries of query blocks rows[0..R)
+    in that order; k: [B, N, Hkv, d] all raw keys.  Same definitions as
+    ``sparse_select`` restricted to those blocks.  Returns (q_hat_rows,
+    k_hat, kbar, idx [B, Hkv, R, W], scores [B, Hkv, R, nb]).
+    """
+    rows = [int(i) for i in rows]
+    qh = rms_norm(q_rows, wq, eps)
+    kh = rms_norm(k, wk, eps)
+    kbar = block_means(kh, block)
+    sd = score_dtype
+    scores = block_scores(_selection_inputs(q_rows, wq, eps, block, sd, qh),
+                          _selection_inputs(k, wk, eps, block, sd, kh), sd, rows=rows)
+    B, Hkv = scores.shape[:2]
+    idx = np.full((B, Hkv, len(rows), topk + n_init + n_local), -1, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            for r, i in enumerate(rows):
+                sel = select_row(scores[b, g, r], i, topk, n_init, n_local)
+                idx[b, g, r, : len(sel)] = sel
     return qh, kh, kbar, idx, scores
 
 
@@ -322,47 +366,67 @@ def sparse_select(q, k, wq, wk, *, block=64, topk=16, n_init=1, n_local=2, eps=1
 # Gathered block-sparse attention
 # ---------------------------------------------------------------------------
 
-def sparse_attention(qh, kh, v, idx, block, scale=None, query_blocks=None):
-    """Exact softmax attention of each query over its selected key blocks.
+def sparse_attention_rows(qh_rows, kh, v, idx_rows, rows, block, scale=None):
+    """Exact softmax attention of the query blocks ``rows`` over their
+    selected key blocks.
 
-    qh: [B, N, Hq, d] normalised queries; kh, v: [B, N, Hkv, d]; idx as from
-    ``select_blocks``.  Query t in block i of head h (kv head h // (Hq/Hkv))
-    attends to every key s in a selected block with s <= t, logits scaled
-    by ``scale`` (default 1/sqrt(d)).  Query blocks outside
-    ``query_blocks`` are left NaN.
+    qh_rows: [B, R*block, Hq, d] normalised queries of blocks rows[0..R) in
+    that order; kh, v: [B, N, Hkv, d]; idx_rows: [B, Hkv, R, W] their index
+    lists (-1 padded).  Query t of block i (= rows[r]) and head h (kv head
+    h // (Hq/Hkv)) attends to every key s in a selected block with s <= t,
+    logits scaled by ``scale`` (default 1/sqrt(d)).  Returns [B, R*block, Hq, dv].
     """
-    qh = np.asarray(qh, F64)
+    qh_rows = np.asarray(qh_rows, F64)
     kh = np.asarray(kh, F64)
     v = np.asarray(v, F64)
-    B, N, Hq, d = qh.shape
+    B, _, Hq, d = qh_rows.shape
     Hkv = kh.shape[2]
     G = Hq // Hkv
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    nb = N // block
-    o = np.full((B, N, Hq, v.shape[-1]), np.nan, dtype=F64)
-    qbs = range(nb) if query_blocks is None else query_blocks
+    o = np.empty((B, len(rows) * block, Hq, v.shape[-1]), dtype=F64)
     for b in range(B):
         for g in range(Hkv):
-            for i in qbs:
-                sel = [int(j) for j in idx[b, g, i] if j >= 0]
+            for r, i in enumerate(rows):
+                sel = [int(j) for j in idx_rows[b, g, r] if j >= 0]
                 pos = np.concatenate([np.arange(j * block, (j + 1) * block) for j in sel])
                 K = kh[b, pos, g]                      # [L, d]
                 V = v[b, pos, g]
                 t = np.arange(i * block, (i + 1) * block)
-                Q = qh[b, i * block:(i + 1) * block, g * G:(g + 1) * G]   # [T, G, d]
+                Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G]   # [T, G, d]
                 logits = np.einsum("tgd,ld->tgl", Q, K) * scale
                 mask = pos[None, :] <= t[:, None]       # [T, L]
                 logits = np.where(mask[:, None, :], logits, -np.inf)
                 m = logits.max(axis=-1, keepdims=True)
                 p = np.exp(logits - m)
                 p = p / p.sum(axis=-1, keepdims=True)
-                o[b, i * block:(i + 1) * block, g * G:(g + 1) * G] = np.einsum("tgl,ld->tgd", p, V)
+                o[b, r * block:(r + 1) * block, g * G:(g + 1) * G] = np.einsum("tgl,ld->tgd", p, V)
+    return o
+
+
+def sparse_attention(qh, kh, v, idx, block, scale=None, query_blocks=None):
+    """Exact softmax attention of each query over its selected key blocks.
+
+    qh: [B, N, Hq, d] normalised queries; kh, v: [B, N, Hkv, d]; idx as from
+    ``select_blocks``.  The definition is ``sparse_attention_rows`` applied
+    to every query block (or to ``query_blocks``); the others are left NaN.
+    """
+    qh = np.asarray(qh, F64)
+    B, N, Hq, d = qh.shape
+    nb = N // block
+    rows = list(range(nb)) if query_blocks is None else [int(i) for i in query_blocks]
+    o = np.full((B, N, Hq, np.shape(v)[-1]), np.nan, dtype=F64)
+    if not rows:
+        return o
+    q_rows = np.concatenate([qh[:, i * block:(i + 1) * block] for i in rows], axis=1)
+    o_rows = sparse_attention_rows(q_rows, kh, v, np.asarray(idx)[:, :, rows], rows, block, scale)
+    for r, i in enumerate(rows):
+        o[:, i * block:(i + 1) * block] = o_rows[:, r * block:(r + 1) * block]
     return o
 
 
 def sparse_layer(q, k, v, g, wq, wk, *, block=64, topk=16, n_init=1, n_local=2,
-                 eps=1e-6, scale=None, score_dtype=np.float32, query_blocks=None):
+                 eps=1e-6, scale=None, score_dtype=F64, query_blocks=None):
     """One sparse SALA layer: QK-RMSNorm without RoPE (NoPE), block selection,
     gathered exact attention, sigmoid output gate.
 
@@ -373,6 +437,21 @@ def sparse_layer(q, k, v, g, wq, wk, *, block=64, topk=16, n_init=1, n_local=2,
         score_dtype=score_dtype, rows=query_blocks)
     o = sparse_attention(qh, kh, v, idx, block, scale, query_blocks)
     return sigmoid(g) * o, (qh, kh, kbar, idx, scores)
+
+
+def sparse_layer_rows(q_rows, g_rows, rows, k, v, wq, wk, *, block=64, topk=16, n_init=1,
+                      n_local=2, eps=1e-6, scale=None, score_dtype=F64):
+    """``sparse_layer`` for the query blocks ``rows`` only: q_rows / g_rows
+    are the raw queries / gate values of those blocks ([B, R*block, Hq, d],
+    in the order of ``rows``); k, v cover the whole sequence.
+
+    Returns (out_rows, (q_hat_rows, k_hat, kbar, idx_rows, scores_rows)).
+    """
+    qh, kh, kbar, idx, scores = sparse_select_rows(
+        q_rows, rows, k, wq, wk, block=block, topk=topk, n_init=n_init, n_local=n_local,
+        eps=eps, score_dtype=score_dtype)
+    o = sparse_attention_rows(qh, kh, v, idx, rows, block, scale)
+    return sigmoid(g_rows) * o, (qh, kh, kbar, idx, scores)
 
 
 # ---------------------------------------------------------------------------
@@ -397,7 +476,7 @@ def decode_linear_step(S, q, k, v, g, lam, wq, wk, pos, *, rope_base=10000.0, ep
 
 
 def decode_sparse_step(k_hist, v_hist, q, g, wq, wk, pos, *, block=64, topk=64, n_init=1,
-                       n_local=4, eps=1e-6, scale=None, score_dtype=np.float32):
+                       n_local=4, eps=1e-6, scale=None, score_dtype=F64):
     """One decode token of the sparse layer at position ``pos``.
 
     k_hist, v_hist: raw keys / values of positions [0, pos] ([B, pos+1, Hkv, d]),

@@ -242,6 +242,55 @@ def check_selection_ties(orc):
     assert [int(j) for j in orc.select_blocks(sc, 50, 1, 2, rows=[9])[0, 0, 9] if j >= 0] == list(range(10))
 
 
+def check_sparse_select_exhaustive(orc):
+    # The whole selection stage on raw inputs against an independent
+    # computation: block means of hand-normalised rows, group-summed queries,
+    # then the best-scoring candidate subset by exhaustive search (fp64).
+    r = _rng(15)
+    B, N, Hq, Hkv, d, blk = 1, 14 * 8, 4, 2, 8, 8
+    q = r.standard_normal((B, N, Hq, d))
+    k = r.standard_normal((B, N, Hkv, d))
+    w = np.ones(d)
+    topk, n_init, n_local = 3, 1, 2
+    _, _, _, idx, _ = orc.sparse_select(q, k, w, w, block=blk, topk=topk, n_init=n_init,
+                                        n_local=n_local)
+    nrm = lambda x: x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + 1e-6)
+    nb = N // blk
+    for g in range(Hkv):
+        kb = [np.mean(nrm(k[0, j * blk:(j + 1) * blk, g]), axis=0) for j in range(nb)]
+        for i in range(nb):
+            qg = sum(np.mean(nrm(q[0, i * blk:(i + 1) * blk, h]), axis=0)
+                     for h in (2 * g, 2 * g + 1))
+            cand = list(range(n_init, i - n_local + 1))
+            best = ()
+            if cand:
+                best = max(itertools.combinations(cand, min(topk, len(cand))),
+                           key=lambda c: sum(float(kb[j] @ qg) for j in c))
+            want = sorted(set(range(min(n_init, i + 1))) | set(range(max(0, i - n_local + 1), i + 1))
+                          | set(best))
+            assert [int(j) for j in idx[0, g, i] if j >= 0] == want, (g, i)
+
+
+def check_sparse_rows_forms(orc):
+    # The row forms compute the same definitions as the full forms on the
+    # chosen query blocks (block numbers, causality and selection included).
+    r = _rng(16)
+    B, N, Hq, Hkv, d, blk = 2, 24 * 16, 6, 2, 16, 16
+    q, g = (r.standard_normal((B, N, Hq, d)) for _ in range(2))
+    k, v = (r.standard_normal((B, N, Hkv, d)) for _ in range(2))
+    w = 1.0 + 0.1 * r.standard_normal(d)
+    kw = dict(block=blk, topk=3, n_init=1, n_local=2)
+    full, (qh, kh, kbar, idx, scores) = orc.sparse_layer(q, k, v, g, w, w, **kw)
+    rows = [23, 0, 9, 4, 17]
+    cat = lambda x: np.concatenate([x[:, i * blk:(i + 1) * blk] for i in rows], axis=1)
+    out, (qh_r, kh_r, kbar_r, idx_r, sc_r) = orc.sparse_layer_rows(cat(q), cat(g), rows, k, v,
+                                                                   w, w, **kw)
+    assert _rel(out, cat(full)) < 1e-13
+    assert np.array_equal(idx_r, idx[:, :, rows])
+    assert np.array_equal(sc_r, scores[:, :, rows])
+    assert _rel(kbar_r, kbar) < 1e-15 and _rel(qh_r, cat(qh)) < 1e-15
+
+
 # --------------------------------------------------------------------------- sparse attention
 
 def _sdpa(q, k, v, mask=None, causal=False, scale=None):
@@ -348,6 +397,7 @@ ALL_CHECKS = [
     check_rope_invariants, check_sigmoid, check_linear_brute_force, check_linear_three_forms,
     check_linear_special_lambdas, check_linear_segments, check_linear_layer_gate_rope,
     check_block_means_and_scores, check_selection_exhaustive, check_selection_ties,
+    check_sparse_select_exhaustive, check_sparse_rows_forms,
     check_sparse_dense_limit, check_sparse_block_diagonal, check_sparse_masked_sdpa,
     check_decode_linear, check_decode_sparse,
 ]

@@ -35,15 +35,21 @@ MUTANTS = [
     ("state transposed", "(Qc @ S)", "(Qc @ S.T[:S.shape[0], :S.shape[1]] if S.shape[0] == S.shape[1] else Qc @ S)"),
     ("gate missing", "state_in, heads)\n    return sigmoid(g) * o, S", "state_in, heads)\n    return o, S"),
     ("scores not scaled", "/ dtype(math.sqrt(d))", "/ dtype(1.0)"),
-    ("group mapping interleaved", "qg = qbar.reshape(B, Hkv, G, nb, d)", "qg = qbar.reshape(B, G, Hkv, nb, d).swapaxes(1, 2)"),
+    ("group mapping interleaved", "qg = qbar.reshape(B, Hkv, G, nq, d)", "qg = qbar.reshape(B, G, Hkv, nq, d).swapaxes(1, 2)"),
     ("tie-break to higher index", "np.lexsort((cand, -sc))", "np.lexsort((-cand, -sc))"),
     ("local window one short", "local = set(range(max(0, b - n_local + 1), b + 1))\n    lo, hi",
      "local = set(range(max(0, b - n_local + 2), b + 1))\n    lo, hi"),
     ("candidates overlap local", "lo, hi = n_init, b - n_local", "lo, hi = n_init, b - 1"),
     ("causal mask off by one", "mask = pos[None, :] <= t[:, None]", "mask = pos[None, :] < t[:, None] + 2"),
-    ("softmax scale missing", "scale = 1.0 / math.sqrt(d)\n    nb = N // block", "scale = 1.0\n    nb = N // block"),
-    ("sparse gqa mapping", "Q = qh[b, i * block:(i + 1) * block, g * G:(g + 1) * G]",
-     "Q = qh[b, i * block:(i + 1) * block, g::Hkv]"),
+    ("softmax scale missing", "scale = 1.0 / math.sqrt(d)\n    o = np.empty(", "scale = 1.0\n    o = np.empty("),
+    ("sparse gqa mapping", "Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G]",
+     "Q = qh_rows[b, r * block:(r + 1) * block, g::Hkv]"),
+    ("row scores ignore the block numbers", "qi = np.arange(nq) if rows is None else np.asarray(rows)",
+     "qi = np.arange(nq)"),
+    ("row attention uses the row number as the block", "t = np.arange(i * block, (i + 1) * block)",
+     "t = np.arange(r * block, (r + 1) * block)"),
+    ("selection ranked on unnormalised queries",
+     "xs = exact if sd is F64 else", "xs = np.asarray(x, sd) if sd is F64 else"),
     ("decode state update order", "S_new = lam[None, :, None, None] * np.asarray(S, F64) + \\\n"
      "        np.einsum(\"bhk,bhv->bhkv\", kh, np.asarray(v, F64))",
      "S_new = lam[None, :, None, None] * (np.asarray(S, F64) + \\\n"
