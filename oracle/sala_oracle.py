@@ -394,13 +394,15 @@ def sparse_attention_rows(qh_rows, kh, v, idx_rows, rows, block, scale=None):
                 V = v[b, pos, g]
                 t = np.arange(i * block, (i + 1) * block)
                 Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G]   # [T, G, d]
-                logits = np.einsum("tgd,ld->tgl", Q, K) * scale
+                T = Q.shape[0]
+                logits = (Q.reshape(T * G, d) @ K.T).reshape(T, G, -1) * scale
                 mask = pos[None, :] <= t[:, None]       # [T, L]
                 logits = np.where(mask[:, None, :], logits, -np.inf)
                 m = logits.max(axis=-1, keepdims=True)
                 p = np.exp(logits - m)
                 p = p / p.sum(axis=-1, keepdims=True)
-                o[b, r * block:(r + 1) * block, g * G:(g + 1) * G] = np.einsum("tgl,ld->tgd", p, V)
+                o[b, r * block:(r + 1) * block, g * G:(g + 1) * G] = \
+                    (p.reshape(T * G, -1) @ V).reshape(T, G, -1)
     return o
 
 
