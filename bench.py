@@ -140,23 +140,45 @@ class ClockSampler:
 class GroupPrefill:
     """Pre-allocated inputs, outputs and workspaces of one layer group."""
 
-    def __init__(self, w: wl.Workload, N: int, dev, sala):
+    def __init__(self, w: wl.Workload, N: int, dev, sala, lean: bool = False):
+        """lean: one output buffer shared by the linear layers, and the sparse
+        layer's normalised Q / K carved out of the linear workspace (the calls
+        run in order on one stream), so that the 1M-token group fits in HBM
+        with every layer's inputs resident."""
         self.w, self.N, self.dev, self.sala = w, N, dev, sala
         ln, sp = w.linear, w.sparse
         B = w.batch
-        self.lin_inputs = [wl.layer_inputs(w, l, dev, seqlen=N) for l in range(w.n_linear)]
+        self.lin_inputs = []
+        for l in range(w.n_linear):
+            self.lin_inputs.append(wl.layer_inputs(w, l, dev, seqlen=N))
+            torch.cuda.empty_cache()
         self.sp_inputs = wl.layer_inputs(w, w.n_linear, dev, seqlen=N)
+        torch.cuda.empty_cache()
         self.lam = torch.tensor(wl.lam_schedule(ln), dtype=torch.float32, device=dev)
         self.wt = wl.rms_weights(ln.head_dim, dev)
-        self.lin_out = [torch.empty_like(x[0]) for x in self.lin_inputs]
+        if lean:
+            shared = torch.empty_like(self.lin_inputs[0][0])
+            self.lin_out = [shared] * w.n_linear
+        else:
+            self.lin_out = [torch.empty_like(x[0]) for x in self.lin_inputs]
         self.ld = sala.linear_desc(B, N, ln.heads, ln.head_dim, ln.chunk, w.torch_dtype)
         self.sd = sala.sparse_desc(B, N, sp.q_heads, sp.kv_heads, sp.head_dim, sp.block, sp.topk,
                                    sp.n_init, sp.n_local, w.torch_dtype)
         self.lws = sala.workspace(sala.sala_linear_workspace_size(self.ld), dev)
         self.sws = sala.workspace(sala.sala_sparse_workspace_size(self.sd), dev)
         nb = N // sp.block
-        self.qn = torch.empty((B, N, sp.q_heads, sp.head_dim), dtype=torch.bfloat16, device=dev)
-        self.kn = torch.empty((B, N, sp.kv_heads, sp.head_dim), dtype=torch.bfloat16, device=dev)
+        nq = B * N * sp.q_heads * sp.head_dim
+        nk = B * N * sp.kv_heads * sp.head_dim
+        if lean and self.lws.numel() >= 2 * (nq + nk) + 256:
+            off = (2 * nq + 255) // 256 * 256
+            self.qn = self.lws[:2 * nq].view(torch.bfloat16).view(B, N, sp.q_heads, sp.head_dim)
+            self.kn = self.lws[off:off + 2 * nk].view(torch.bfloat16).view(B, N, sp.kv_heads,
+                                                                           sp.head_dim)
+        else:
+            self.qn = torch.empty((B, N, sp.q_heads, sp.head_dim), dtype=torch.bfloat16,
+                                  device=dev)
+            self.kn = torch.empty((B, N, sp.kv_heads, sp.head_dim), dtype=torch.bfloat16,
+                                  device=dev)
         self.kbar = torch.empty((B, nb, sp.kv_heads, sp.head_dim), dtype=torch.float32, device=dev)
         self.idx = torch.empty((B, sp.kv_heads, nb, sala.sala_sparse_index_width(self.sd)),
                                dtype=torch.int32, device=dev)
@@ -267,24 +289,35 @@ def replica_throughput(tokens_per_rank_step: int, steps: int, max_ms: float, ws:
     return tokens_per_rank_step * ws * steps / (max_ms / 1e3)
 
 
-def cpu_baseline_sample(w: wl.Workload, budget_s: float = 20.0):
-    """Time the oracle as it stands on a bounded sample of the workload.
+CPU_SAMPLE_TOKENS = 4096        # linear layer: tokens of the timed sample (all heads)
+CPU_SAMPLE_BLOCKS = 8           # sparse layer: query blocks of the timed sample
 
-    Linear part: one linear layer, all heads, over the first T tokens (work per
-    token is constant).  Sparse part: the last q query blocks of a sequence of
-    Ns tokens (their selection is full).  Returns tokens/s of a layer group
-    extrapolated by work, the thread count and a description.
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline_sample(w: wl.Workload):
+    """Time the oracle as it stands on one bounded sample of the workload
+    (the same sample in both arms of the benchmark).
+
+    Linear part: one linear layer, all heads, over the first
+    CPU_SAMPLE_TOKENS tokens (its work per token is constant).  Sparse part:
+    the last CPU_SAMPLE_BLOCKS query blocks of a sequence long enough that
+    they take the full top-k selection, through the oracle's row form (only
+    those blocks' queries are normalised; every key is, as the selection
+    needs).  Returns layer-group tokens/s extrapolated by per-token work, the
+    thread count, a description and the seconds the sample took.
     """
     import numpy as np
     import oracle
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        threads = len(os.sched_getaffinity(0))
     ln, sp = w.linear, w.sparse
     f64 = lambda t: t.to(torch.float64).numpy()
-    T = 512 if budget_s < 15 else 4096
+    T = CPU_SAMPLE_TOKENS
     q, k, v, g = (f64(x) for x in wl.layer_inputs(w, 0, "cpu", seqlen=T))
     lam = np.asarray(wl.lam_schedule(ln))
     wt = np.ones(ln.head_dim)
@@ -293,19 +326,117 @@ def cpu_baseline_sample(w: wl.Workload, budget_s: float = 20.0):
     t_lin = (time.perf_counter() - t0) / T
     need = (sp.topk + sp.n_init + sp.n_local) * sp.block
     Ns = max(4096, 2 * need)
-    nq = 2 if budget_s < 15 else 8
+    nq = CPU_SAMPLE_BLOCKS
     nb = Ns // sp.block
+    rows = list(range(nb - nq, nb))
     q, k, v, g = (f64(x) for x in wl.layer_inputs(w, w.n_linear, "cpu", seqlen=Ns))
+    cat = lambda x: np.concatenate([x[:, i * sp.block:(i + 1) * sp.block] for i in rows], axis=1)
     t0 = time.perf_counter()
-    oracle.sparse_layer(q, k, v, g, wt, wt, block=sp.block, topk=sp.topk, n_init=sp.n_init,
-                        n_local=sp.n_local, query_blocks=list(range(nb - nq, nb)))
+    oracle.sparse_layer_rows(cat(q), cat(g), rows, k, v, wt, wt, block=sp.block, topk=sp.topk,
+                             n_init=sp.n_init, n_local=sp.n_local)
     t_sp = (time.perf_counter() - t0) / (nq * sp.block)
     per_token = w.n_linear * t_lin + t_sp
     desc = (f"oracle (numpy fp64) on host cores: linear layer x{w.n_linear} timed on 1 layer x "
             f"{ln.heads} heads x {T} tokens; sparse layer timed on the last {nq} query blocks "
-            f"of a {Ns}-token sequence (full top-{sp.topk} selection, scoring the whole prefix); "
-            f"tokens/s of the group extrapolated by per-token work")
-    return 1.0 / per_token, threads, desc, t_lin * T + t_sp * nq * sp.block
+            f"of a {Ns}-token sequence (full top-{sp.topk} selection over every earlier block); "
+            f"layer-group tokens/s extrapolated by per-token work")
+    return 1.0 / per_token, cpu_threads(), desc, t_lin * T + t_sp * nq * sp.block
+
+
+def config_of(w: wl.Workload, N: int, ws: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": w.name, "seq_len": N, "batch": w.batch,
+            "layers": f"{w.n_linear} linear + 1 sparse",
+            "heads": w.linear.heads, "kv_heads": w.sparse.kv_heads,
+            "head_dim": w.linear.head_dim, "chunk": w.linear.chunk,
+            "block": w.sparse.block, "topk": w.sparse.topk,
+            "n_init": w.sparse.n_init, "n_local": w.sparse.n_local,
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": "inputs larger than L2 (no flush needed)"}
+
+
+def time_group(w: wl.Workload, N: int, dev, sala, steps: int, warmup: int, ws: int = 1,
+               lean: bool = False, clocks=None):
+    """Warm up, then time `steps` group steps with CUDA events on the
+    launching stream (barrier + synchronize on both sides).  Returns the
+    GroupPrefill, the max-over-ranks elapsed ms, per-call event times and
+    the number of library launches in the timed region."""
+    grp = GroupPrefill(w, N, dev, sala, lean=lean)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        grp.step()
+    torch.cuda.synchronize()
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    if clocks is not None:
+        clocks.start()
+    barrier(ws)
+    torch.cuda.synchronize()
+    launches0 = sala.sala_kernel_launch_count()
+    timed = []
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        grp.step(timed)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop() if clocks is not None else None
+    launches = sala.sala_kernel_launch_count() - launches0
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), ws)
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    per_call = {}
+    for name, e0, e1 in timed:
+        per_call.setdefault(name, []).append(e0.elapsed_time(e1))
+    return grp, elapsed_ms, per_call, launches, clk
+
+
+def call_rooflines(w: wl.Workload, N: int, per_call: dict, steps: int, peaks: dict) -> dict:
+    """Per-call achieved work against the measured peaks.  The calls are
+    timed in windows of milliseconds inside a sub-second region, so the
+    tensor-bound call is rated against the burst bf16 peak (the sustained
+    figure is given beside it)."""
+    work = {
+        "linear_prefill": ("hbm", linear_bytes(w, N)),
+        "sparse_select": ("hbm", select_bytes(w, N)),
+        "sparse_prefill": ("tensor", sparse_attn_flops(w, N)),
+    }
+    calls = {}
+    for name, ts in per_call.items():
+        avg = sum(ts) / len(ts)
+        bound, amount = work[name]
+        c = {"ms": round(avg, 4), "launches_per_step": len(ts) // steps, "bound": bound}
+        if bound == "hbm":
+            ach = amount / (avg / 1e3) / 1e9
+            c.update(achieved=round(ach, 2), peak=peaks["hbm_gbs"], unit="GB/s",
+                     frac=round(ach / peaks["hbm_gbs"], 4))
+        else:
+            ach = amount / (avg / 1e3) / 1e12
+            c.update(achieved=round(ach, 2), peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                     frac=round(ach / peaks["bf16_tflops"], 4),
+                     frac_of_sustained=round(ach / peaks["bf16_tflops_sustained"], 4))
+        calls[name] = c
+    tot = sum(c["ms"] * c["launches_per_step"] for c in calls.values())
+    for c in calls.values():
+        c["share"] = round(c["ms"] * c["launches_per_step"] / tot, 4)
+    return calls
+
+
+def per_config_entry(w, N, elapsed_ms, steps, per_call, peaks, ws, note=None):
+    calls = call_rooflines(w, N, per_call, steps, peaks)
+    ms = elapsed_ms / steps
+    e = {"workload": w.name, "seq_len": N, "topk": w.sparse.topk, "steps": steps,
+         "ms_per_step": round(ms, 4),
+         "tokens_per_s": round(replica_throughput(w.batch * N, steps, elapsed_ms, ws), 1),
+         "calls": calls}
+    if note:
+        e["note"] = note
+    return e
+
+
+PER_CONFIG = [("group_32k", 10, False), ("group_128k", 5, False), ("group_1m", 3, True)]
 
 
 def run_ours(args):
@@ -316,83 +447,57 @@ def run_ours(args):
     w = wl.WORKLOADS[args.workload]
     N = args.seqlen or w.seqlen
     peaks, peak_kind = load_peaks()
-    grp = GroupPrefill(w, N, dev, sala)
-    torch.cuda.synchronize()
-
-    for _ in range(args.warmup):
-        grp.step()
-    torch.cuda.synchronize()
-    if sala.sala_get_device_status() != 0:
-        raise RuntimeError("device status word set during warm-up")
-
     clocks = ClockSampler(local)
-    clocks.start()
-    barrier(ws)
-    torch.cuda.synchronize()
-    launches0 = sala.sala_kernel_launch_count()
-    timed = []
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(args.steps):
-        grp.step(timed)
-    end.record()
-    torch.cuda.synchronize()
-    barrier(ws)
-    clk = clocks.stop()
-    launches = sala.sala_kernel_launch_count() - launches0
-    elapsed_ms = max_over_ranks(start.elapsed_time(end), ws)
-    if sala.sala_get_device_status() != 0:
-        raise RuntimeError("device status word set during the timed region")
-    per_call = {}
-    for name, e0, e1 in timed:
-        per_call.setdefault(name, []).append(e0.elapsed_time(e1))
+    grp, elapsed_ms, per_call, launches, clk = time_group(w, N, dev, sala, args.steps,
+                                                          args.warmup, ws, clocks=clocks)
     ms_per_step = elapsed_ms / args.steps
     value = replica_throughput(w.batch * N, args.steps, elapsed_ms, ws)
-
-    # per-call roofline (dominant call reported as "roofline")
-    calls = {}
-    work = {
-        "linear_prefill": ("hbm", linear_bytes(w, N)),
-        "sparse_select": ("hbm", select_bytes(w, N)),
-        "sparse_prefill": ("tensor", sparse_attn_flops(w, N)),
-    }
-    for name, ts in per_call.items():
-        avg = sum(ts) / len(ts)
-        bound, amount = work[name]
-        if bound == "hbm":
-            ach, pk, unit = amount / (avg / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
-        else:
-            ach, pk, unit = amount / (avg / 1e3) / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s"
-        calls[name] = {"ms": round(avg, 4), "launches_per_step": ts and len(ts) // args.steps,
-                       "bound": bound, "achieved": round(ach, 2), "peak": pk, "unit": unit,
-                       "frac": round(ach / pk, 4), "share": 0.0}
-    tot = sum(c["ms"] * c["launches_per_step"] for c in calls.values())
-    for c in calls.values():
-        c["share"] = round(c["ms"] * c["launches_per_step"] / tot, 4)
+    calls = call_rooflines(w, N, per_call, args.steps, peaks)
     dom = max(calls, key=lambda n: calls[n]["share"])
     traffic = kernel_traffic(args.workload, dom)
     d = calls[dom]
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
                 "unit": d["unit"], "frac": d["frac"], "traffic": traffic, "kernel": dom,
-                "peak_source": f"{peak_kind} ({'sustained bf16' if d['bound'] == 'tensor' else 'HBM copy'})"}
+                "peak_source": f"{peak_kind} ({'burst bf16' if d['bound'] == 'tensor' else 'HBM copy'})"}
+    if "frac_of_sustained" in d:
+        roofline["frac_of_sustained"] = d["frac_of_sustained"]
 
     # end to end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(grp, args, ws)
+    del grp
+    torch.cuda.empty_cache()
+
+    # the other layer-group workloads (parity cases at their own sizes)
+    per_config = {w.name: per_config_entry(w, N, elapsed_ms, args.steps, per_call, peaks, ws)}
+    if not args.no_per_config:
+        for name, steps, lean in PER_CONFIG:
+            if name == w.name:
+                continue
+            wc = wl.WORKLOADS[name]
+            g2, el, pc, _, _ = time_group(wc, wc.seqlen, dev, sala, steps, 3, ws, lean=lean)
+            del g2
+            torch.cuda.empty_cache()
+            note = ("one output buffer shared by the three linear layers and the sparse "
+                    "layer's normalised Q/K in the linear workspace (memory)") if lean else None
+            per_config[name] = per_config_entry(wc, wc.seqlen, el, steps, pc, peaks, ws, note)
 
     dec = None
     if args.decode_steps > 0:
-        del grp
-        torch.cuda.empty_cache()
         dec = run_decode(wl.WORKLOADS["group_1m"], args.decode_steps, dev, sala, peaks, ws)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        v, threads, desc, secs = cpu_baseline_sample(w, args.cpu_budget)
-        cpu = {"value": round(v, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc, "sample_seconds": round(secs, 2)}
+        vals, threads, desc, secs = [], 1, "", 0.0
+        for _ in range(args.cpu_samples):
+            v, threads, desc, s_ = cpu_baseline_sample(w)
+            vals.append(v)
+            secs += s_
+        cpu = {"value": round(len(vals) / sum(1.0 / v for v in vals), 2), "unit": UNIT,
+               "cores": threads, "kind": "oracle",
+               "sample": desc + f"; {len(vals)} samples, harmonic mean",
+               "sample_seconds": round(secs, 2)}
 
     if rank == 0:
         out = {
@@ -400,19 +505,12 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic N(0,1) inputs, seeded (no trained weights)",
-            "config": {"workload": w.name, "seq_len": N, "batch": w.batch,
-                       "layers": f"{w.n_linear} linear + 1 sparse",
-                       "heads": w.linear.heads, "kv_heads": w.sparse.kv_heads,
-                       "head_dim": w.linear.head_dim, "chunk": w.linear.chunk,
-                       "block": w.sparse.block, "topk": w.sparse.topk,
-                       "n_init": w.sparse.n_init, "n_local": w.sparse.n_local,
-                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (no flush needed)"},
+            "config": config_of(w, N, ws),
             "roofline": roofline, "calls": calls,
             "tensor_frac_of_step": round(sparse_attn_flops(w, N) / (ms_per_step / 1e3) / 1e12
-                                         / peaks["bf16_tflops_sustained"], 4),
+                                         / peaks["bf16_tflops"], 4),
             "e2e": e2e, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
-            "decode": dec,
+            "per_config": per_config, "decode": dec,
         }
         print(json.dumps(out), flush=True)
     if ws > 1:
@@ -500,8 +598,12 @@ def run_decode(w: wl.Workload, steps: int, dev, sala, peaks, ws):
 
 
 def run_e2e(grp: GroupPrefill, args, ws):
-    """Same step through the C ABI, inputs copied from pinned host memory and
-    outputs read back inside the timed region."""
+    """Same step through the C ABI with host buffers: every layer's inputs
+    are copied from pinned host memory and every layer's output read back
+    inside the timed region.  Copies run on two side streams so that the
+    host-to-device copy of layer l+1 and the read-back of layer l-1 overlap
+    the computation of layer l (PCIe is full duplex); events order each
+    buffer's reuse across layers and steps."""
     w, N = grp.w, grp.N
     host_in = []
     for tens in grp.lin_inputs + [grp.sp_inputs]:
@@ -512,30 +614,62 @@ def run_e2e(grp: GroupPrefill, args, ws):
     h2d = sum(t.numel() * t.element_size() for ts in host_in for t in ts)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     steps = max(1, min(args.steps, args.e2e_steps))
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    calls = grp.calls()
+    # layer l = calls of linear layer l; the sparse layer is select + prefill
+    layers = [[c] for c in calls[:w.n_linear]] + [calls[w.n_linear:]]
+    n = len(layers)
+    read_done = [None] * n      # compute finished reading layer l's inputs
+    out_done = [None] * n       # read-back of layer l's output finished
 
     def one():
-        for hs, ds in zip(host_in, dev_in):
-            for h, d in zip(hs, ds):
-                d.copy_(h, non_blocking=True)
-        grp.step()
-        for d, h in zip(dev_out, host_out):
-            h.copy_(d, non_blocking=True)
+        ev_in = []
+        for l in range(n):
+            with torch.cuda.stream(s_in):
+                if read_done[l] is not None:
+                    s_in.wait_event(read_done[l])
+                for h, d in zip(host_in[l], dev_in[l]):
+                    d.copy_(h, non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_in)
+                ev_in.append(e)
+        for l in range(n):
+            comp.wait_event(ev_in[l])
+            if out_done[l] is not None:
+                comp.wait_event(out_done[l])
+            for name, fn in layers[l]:
+                st = fn()
+                if st != 0:
+                    raise RuntimeError(f"{name}: {grp.sala.status_string(st)}")
+            e = torch.cuda.Event()
+            e.record(comp)
+            read_done[l] = e
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e)
+                host_out[l].copy_(dev_out[l], non_blocking=True)
+                e2 = torch.cuda.Event()
+                e2.record(s_out)
+                out_done[l] = e2
 
     one()
     torch.cuda.synchronize()
     barrier(ws)
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record()
+    s.record(comp)
+    s_in.wait_event(s)
     for _ in range(steps):
         one()
-    e.record()
+    comp.wait_stream(s_out)
+    e.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), ws)
     barrier(ws)
     return {"value": round(w.batch * N * ws * steps / (ms / 1e3), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3)}
+            "ms_per_step": round(ms / steps, 3),
+            "overlap": "H2D of layer l+1 and D2H of layer l-1 overlap layer l"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -545,11 +679,13 @@ def run_reference(args):
     if rank != 0:
         return
     w = wl.WORKLOADS[args.workload]
+    N = args.seqlen or w.seqlen
     for _ in range(args.warmup):
-        cpu_baseline_sample(w, budget_s=5.0)
+        cpu_baseline_sample(w)
     vals, secs = [], 0.0
+    threads, desc = 1, ""
     for _ in range(args.steps):
-        v, threads, desc, s = cpu_baseline_sample(w, budget_s=5.0)
+        v, threads, desc, s = cpu_baseline_sample(w)
         vals.append(v)
         secs += s
     value = len(vals) / sum(1.0 / v for v in vals)
@@ -557,14 +693,14 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         # time the oracle would take for one whole step (extrapolated by work)
-        "warmup": args.warmup, "ms_per_step": round(w.batch * w.seqlen / value * 1e3, 1),
+        "warmup": args.warmup, "ms_per_step": round(w.batch * N / value * 1e3, 1),
         "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic N(0,1) inputs, seeded (no trained weights)",
-        "config": {"workload": w.name, "seq_len": w.seqlen, "batch": w.batch,
-                   "layers": f"{w.n_linear} linear + 1 sparse"},
+        "config": config_of(w, N, 1),
         "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads,
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "sample": desc + "; one sample per step",
+                         "sample_seconds": round(secs, 2)},
         "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -582,7 +718,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--cpu-samples", type=int, default=4,
+                    help="oracle samples timed for cpu_baseline (a few seconds each)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other layer-group workloads")
     ap.add_argument("--decode-steps", type=int, default=256,
                     help="decode tokens timed after a 1M-token prefill (0: skip)")
     args = ap.parse_args()

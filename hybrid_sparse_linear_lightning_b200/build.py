@@ -1,7 +1,9 @@
 """Build libsala.so in-tree with nvcc for sm_100a (no GPU needed to compile)."""
 from __future__ import annotations
 
+import json
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -15,7 +17,7 @@ SOURCES = ["api.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-    "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills",
+    "--expt-relaxed-constexpr",
 ]
 
 
@@ -34,19 +36,62 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in deps if os.path.isfile(p))
 
 
+# Kernels whose in-kernel register reallocation (setmaxnreg) is sized for a
+# fixed launch allocation: the build fails unless ptxas gave each exactly
+# this many registers per thread, so a library that built cannot hang on a
+# register split larger than its launch allocation.
+REGISTER_SPLIT_KERNELS = {"linear_segout_kernel": 128}
+REPORT = os.path.join(PKG, "libsala.ptxas.json")
+
+
+def parse_ptxas(text: str) -> dict:
+    """{mangled kernel name: registers per thread} from `ptxas -v` output."""
+    regs, cur = {}, None
+    for line in text.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            cur = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur:
+            regs[cur] = int(m.group(1))
+            cur = None
+    return regs
+
+
+def check_register_splits(regs: dict) -> None:
+    for short, want in REGISTER_SPLIT_KERNELS.items():
+        got = {k: v for k, v in regs.items() if short in k}
+        if not got:
+            raise RuntimeError(f"ptxas report has no entry for {short}")
+        bad = {k: v for k, v in got.items() if v != want}
+        if bad:
+            raise RuntimeError(f"{short}: built with {sorted(set(bad.values()))} registers per "
+                               f"thread; its register split needs exactly {want}")
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not needs_build():
         return LIB
-    cmd = [nvcc_path(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
+    cmd = [nvcc_path(), *NVCC_FLAGS, "-Xptxas", "-v", *extra, "-I", os.path.join(ROOT, "include"),
            "-o", LIB + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        raise subprocess.CalledProcessError(r.returncode, cmd)
+    for line in (r.stdout + r.stderr).splitlines():
+        if re.search(r"[1-9]\d* bytes spill", line) or "warning" in line.lower():
+            sys.stderr.write(line + "\n")
+    regs = parse_ptxas(r.stdout + r.stderr)
+    check_register_splits(regs)
+    with open(REPORT, "w") as f:
+        json.dump({"registers_per_thread": regs}, f, indent=1, sort_keys=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
+    build(force="--force" in sys.argv, verbose=True)
     print(LIB)

@@ -232,10 +232,17 @@ sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
   const size_t smem_b = LsOutLayout::kBytes + 1024;
   auto kern = linear_segout_kernel<__nv_bfloat16>;
   if (allow_smem(kern, smem_b) != cudaSuccess) return SALA_ERR_CUDA;
-  // the in-kernel register split assumes this launch allocation exactly
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SALA_ERR_CUDA;
-  if (fa.numRegs != kLsOutRegsLaunch) return SALA_ERR_UNSUPPORTED;
+  // The in-kernel register split assumes this launch allocation exactly.
+  // The build refuses to produce a library where it differs; this cached
+  // check only keeps a library built some other way from launching a split
+  // larger than its allocation (which would never finish).
+  static std::atomic<int> regs_ok{0};   // 0 unknown, 1 matches, 2 differs
+  if (regs_ok.load(std::memory_order_relaxed) == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SALA_ERR_CUDA;
+    regs_ok.store(fa.numRegs == kLsOutRegsLaunch ? 1 : 2, std::memory_order_relaxed);
+  }
+  if (regs_ok.load(std::memory_order_relaxed) != 1) return SALA_ERR_UNSUPPORTED;
   kern<<<grid, kLsOutThreads, smem_b, st>>>(qm, km, vm, gm, static_cast<const __nv_bfloat16*>(gate),
                                             lambda, seg_state, static_cast<__nv_bfloat16*>(out),
                                             d->seqlen, d->heads, p.seg_tiles, p.n_seg, d->scale);

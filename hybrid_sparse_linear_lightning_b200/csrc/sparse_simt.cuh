@@ -51,6 +51,9 @@ sparse_attn_simt_kernel(const __nv_bfloat16* __restrict__ qn, const __nv_bfloat1
     if (j > i) set_status(kStatusBounds);
     ++nsel;
   }
+  // a valid row lists at least the query's own block; rows with no visible
+  // key get a zero output and the bounds bit
+  if (nsel == 0 && tid == 0) set_status(kStatusBounds);
   __syncthreads();
 
   const int rows = BLK * G;
@@ -123,7 +126,7 @@ sparse_attn_simt_kernel(const __nv_bfloat16* __restrict__ qn, const __nv_bfloat1
       if (r >= rows) continue;
       const int t = r / G, h = g * G + r % G;
       const long long off = (((long long)b * N + (long long)i * BLK + t) * Hq + h) * D;
-      const float inv = 1.f / l[rr];
+      const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;
 #pragma unroll
       for (int e = 0; e < DL; ++e) {
         const int d = lane + 32 * e;

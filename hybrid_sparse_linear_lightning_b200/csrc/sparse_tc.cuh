@@ -121,6 +121,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       sel[n++] = j;
       prev = j;
     }
+    // a valid row lists at least the query's own block; an empty row gets a
+    // zero output and the bounds bit
+    if (n == 0) set_status(kStatusBounds);
     *n_sel_slot = n;
   }
   if (warp == 2) {
@@ -308,7 +311,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     if (ok)
       ok = __all_sync(0xffffffffu,
                       tc::mbar_wait(o_done + 2 * t + ((n_sel - 1) & 1), ((n_sel - 1) >> 1) & 1));
-    if (ok) {
+    if (n_sel == 0) {
+      const int head = hbase + 2 * t + (r >> 6);
+      const long long off = (((long long)b * N + (long long)i * 64 + tok) * Hq + head) * D;
+      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int c = 0; c < D; c += 8) store8(out + off + c, z);
+    } else if (ok) {
       tc::tc_fence_after();
       const int head = hbase + 2 * t + (r >> 6);
       const long long off = (((long long)b * N + (long long)i * 64 + tok) * Hq + head) * D;

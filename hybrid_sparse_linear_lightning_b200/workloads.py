@@ -153,16 +153,20 @@ def layer_inputs(w: Workload, layer: int, device="cpu", seqlen: Optional[int] = 
         d = w.linear.head_dim
     else:
         hq, hk, d = w.sparse.q_heads, w.sparse.kv_heads, w.sparse.head_dim
-    out = []
-    for heads in (hq, hk, hk, hq):
-        out.append(torch.randn((B, N, heads, d), generator=g, device=device,
-                               dtype=torch.float32))
-    if w.salient_key_frac > 0:
-        g2 = _gen(device, 1 + 100 * layer)
-        mask = torch.rand((B, N, hk, 1), generator=g2, device=device) < w.salient_key_frac
-        out[1] = torch.where(mask, out[1] * w.salient_key_mult, out[1])
     dt = w.torch_dtype
-    return [t.to(dt) for t in out]
+    out = []
+    # each tensor is cast as soon as it is drawn (same values as drawing all
+    # four first: the draws come from one generator in the same order), so
+    # at most one fp32 tensor is alive at a time
+    for which, heads in enumerate((hq, hk, hk, hq)):
+        t = torch.randn((B, N, heads, d), generator=g, device=device, dtype=torch.float32)
+        if which == 1 and w.salient_key_frac > 0:
+            g2 = _gen(device, 1 + 100 * layer)
+            mask = torch.rand((B, N, hk, 1), generator=g2, device=device) < w.salient_key_frac
+            t = torch.where(mask, t * w.salient_key_mult, t)
+        out.append(t.to(dt))
+        del t
+    return out
 
 
 def decode_inputs(w: Workload, step: int, device="cpu"):

@@ -67,7 +67,7 @@ def test_reference_arm_line_rank0(capsys):
     import types
     import bench
     os.environ.pop("RANK", None)
-    bench.run_reference(types.SimpleNamespace(workload="group_256k", steps=1, warmup=0))
+    bench.run_reference(types.SimpleNamespace(workload="group_256k", seqlen=0, steps=1, warmup=0))
     line = capsys.readouterr().out.strip().splitlines()[-1]
     d = json.loads(line)
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
