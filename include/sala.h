@@ -130,7 +130,11 @@ sala_status sala_sparse_select(const sala_sparse_desc* d, const void* q, const v
  *     SALA_ERR_WORKSPACE and launch nothing.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current and caches it; make
- *     that first call before any stream capture on the device.
+ *     that first call before any stream capture on the device.  The cached
+ *     address belongs to the device's context as it was then: after
+ *     cudaDeviceReset (or anything else that destroys and recreates that
+ *     context) the cache is stale, so do not call this entry point again in
+ *     a process that reset the device.
  *   - The library calls no cudaMalloc / cudaFree here.
  *   - All calls on one device share the array, so calls that may overlap on
  *     the GPU (different streams without ordering) race and must not be

@@ -276,3 +276,40 @@ def test_decode_steps(sala):
     for l in range(w.n_linear):
         assert rel_err(f64(states[l]), ref_states[l]) <= TOL
     assert sala.sala_get_device_status() == 0
+
+
+@pytest.mark.parametrize("name,seqlen", [("group_32k", 1024), ("tiny_2k_f32", 1024)])
+def test_sparse_prefill_empty_index_row(sala, name, seqlen):
+    """An index row that lists no block (first entry -1) is an argument error
+    caught on the device: that row's output is zero, the bounds bit is set,
+    and every other row is computed as usual.  Covers the tensor-core kernel
+    (bf16, 16 q heads per kv head) and the CUDA-core one (fp32)."""
+    dev = torch.device("cuda")
+    w = wl.WORKLOADS[name]
+    sp = w.sparse
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev, seqlen=seqlen)
+    wt = wl.rms_weights(sp.head_dim, dev)
+    qn, kn, kbar, idx = sala.sparse_select(q, k, wt, wt, block=sp.block, topk=sp.topk,
+                                           n_init=sp.n_init, n_local=sp.n_local)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == sala.SALA_OK
+    bad = 5
+    idx[0, 0, bad, :] = -1
+    out = sala.sparse_prefill(qn, kn, v, g, idx, block=sp.block, topk=sp.topk, n_init=sp.n_init,
+                              n_local=sp.n_local)
+    assert sala.sala_get_device_status() == sala.SALA_ERR_DEVICE_FAULT
+    assert sala.sala_get_device_status() == sala.SALA_OK          # read clears the word
+    G = sp.q_heads // sp.kv_heads
+    rows = slice(bad * sp.block, (bad + 1) * sp.block)
+    assert torch.count_nonzero(out[:, rows, :G]) == 0
+    gidx = idx.cpu().numpy()
+    # reference: the bad row of kv head 0 borrows kv head 1's list (when there
+    # is one) so the oracle runs; those heads are then skipped in the compare
+    ref_idx = gidx.copy()
+    ref_idx[0, 0, bad] = gidx[0, -1, bad] if sp.kv_heads > 1 else -1
+    blocks = [i for i in range(seqlen // sp.block) if sp.kv_heads > 1 or i != bad]
+    want = oracle.sigmoid(f64(g)) * oracle.sparse_attention(
+        oracle.rms_norm(f64(q), f64(wt)), oracle.rms_norm(f64(k), f64(wt)), f64(v), ref_idx,
+        sp.block, query_blocks=blocks)
+    want[:, rows, :G] = 0.0
+    assert rel_err(f64(out), want) <= TOL

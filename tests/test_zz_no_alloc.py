@@ -11,7 +11,6 @@ import pytest
 import torch
 
 from hybrid_sparse_linear_lightning_b200 import workloads as wl
-from tests.parity import TOL, f64, rel_err
 
 sala = pytest.importorskip("hybrid_sparse_linear_lightning_b200.sala")
 
@@ -51,7 +50,8 @@ def test_noalloc_matches_workspace_select_on_two_calls(cuda_device):
         ref, got = _run_both(wl.WORKLOADS[name], seqlen)
         qn, kn, kbar, idx = ref
         gq, gk, gkbar, gidx = got
-        assert rel_err(f64(gq), f64(qn)) <= TOL
-        assert rel_err(f64(gk), f64(kn)) <= TOL
-        assert rel_err(f64(gkbar), f64(kbar)) <= TOL
+        # same kernels on the same inputs: identical bits, scratch location aside
+        assert torch.equal(gq, qn)
+        assert torch.equal(gk, kn)
+        assert torch.equal(gkbar, kbar)
         assert torch.equal(gidx, idx)
