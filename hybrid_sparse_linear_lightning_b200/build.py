@@ -81,9 +81,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise subprocess.CalledProcessError(r.returncode, cmd)
+    cur = ""
     for line in (r.stdout + r.stderr).splitlines():
+        m = re.search(r"Function properties for (\S+)", line)
+        if m:
+            cur = m.group(1)
         if re.search(r"[1-9]\d* bytes spill", line) or "warning" in line.lower():
-            sys.stderr.write(line + "\n")
+            sys.stderr.write(f"{cur}: {line.strip()}\n")
     regs = parse_ptxas(r.stdout + r.stderr)
     check_register_splits(regs)
     with open(REPORT, "w") as f:

@@ -292,31 +292,27 @@ sala_status run_sparse_prefill(const sala_sparse_desc* d, const void* qn, const 
 }
 
 struct DecodeWs {
-  size_t qhat, cand_key, cand_idx, idx, part, counters, total;
+  size_t ctl, hist, thr, keys, above, bnd, idx, qhat, part, total, zero_bytes;
 };
-constexpr int kDecodeMergeMax = 8192;   // candidates entering the exact merge
 DecodeWs decode_ws(const sala_decode_desc* d) {
   const sala_sparse_desc& s = d->sp;
   const size_t B = s.batch, Hq = s.q_heads, Hkv = s.kv_heads, D = s.head_dim;
+  const size_t BG = B * Hkv, G = Hq / Hkv;
   const size_t width = s.topk + s.n_init + s.n_local;
+  const size_t capb = (size_t)(d->cache_capacity / s.block);
   DecodeWs w;
-  w.qhat = 0;
-  w.cand_key = w.qhat + align_up(B * Hq * D * 4);
-  w.cand_idx = w.cand_key + align_up(B * Hkv * kDecodeMergeMax * 4);
-  w.idx = w.cand_idx + align_up(B * Hkv * kDecodeMergeMax * 4);
-  w.part = w.idx + align_up(B * Hkv * width * 4);
-  w.counters = w.part + align_up(B * Hkv * width * (Hq / Hkv) * (D + 4) * 4);
-  w.total = w.counters + align_up(B * Hkv * 2 * 4);
+  w.ctl = 0;
+  w.hist = w.ctl + align_up(dec_ctl_words((int)BG) * 4);
+  w.thr = w.hist + align_up(BG * kDecBins * 4);
+  w.zero_bytes = w.thr;                          // control words and histograms
+  w.keys = w.thr + align_up(BG * 4);
+  w.above = w.keys + align_up(BG * capb * 4);
+  w.bnd = w.above + align_up(BG * std::max<size_t>(s.topk, 1) * 4);
+  w.idx = w.bnd + align_up(BG * kDecBndMax * 8);
+  w.qhat = w.idx + align_up(BG * width * 4);
+  w.part = w.qhat + align_up(B * Hq * D * 4);
+  w.total = w.part + align_up(BG * width * G * (D + 4) * 4);
   return w;
-}
-
-// Candidate chunk of the decode selection: 256 blocks, doubled until the
-// local lists (chunks x k) fit the exact merge.
-void decode_chunks(int n_cand, int k, int* chunk, int* n_chunks) {
-  int c = 256;
-  while (k > 0 && (long long)((n_cand + c - 1) / c) * k > kDecodeMergeMax) c *= 2;
-  *chunk = c;
-  *n_chunks = n_cand > 0 ? (n_cand + c - 1) / c : 1;
 }
 
 sala_status check_decode(const sala_decode_desc* d) {
@@ -338,74 +334,79 @@ sala_status check_decode(const sala_decode_desc* d) {
   return SALA_OK;
 }
 
-template <typename T, int DL, int DS>
+// SMs of the current device (cached per device).
+int device_sms() {
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  return sms[dev];
+}
+
+template <typename T, int D>
 sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void* k_cache,
                        void* v_cache, float* kbar, float* ksum, int64_t cur_len, char* ws,
                        cudaStream_t st) {
-  static_assert(DL == DS, "one head_dim for the group");
-  constexpr int D = DS;
   const sala_linear_desc& L = d->lin;
   const sala_sparse_desc& S = d->sp;
-  const int sl = d->n_linear;
   const DecodeWs w = decode_ws(d);
-  DecodeLinearArgs a;
-  memset(&a, 0, sizeof(a));
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
   for (int l = 0; l < d->n_linear; ++l) {
-    a.q[l] = io->q[l]; a.k[l] = io->k[l]; a.v[l] = io->v[l]; a.gate[l] = io->gate[l];
-    a.wq[l] = io->wq[l]; a.wk[l] = io->wk[l]; a.lambda[l] = io->lambda[l];
-    a.state[l] = io->lin_state[l]; a.out[l] = io->out[l];
+    p.lq[l] = io->q[l]; p.lk[l] = io->k[l]; p.lv[l] = io->v[l]; p.lgate[l] = io->gate[l];
+    p.lwq[l] = io->wq[l]; p.lwk[l] = io->wk[l]; p.llam[l] = io->lambda[l];
+    p.lstate[l] = io->lin_state[l]; p.lout[l] = io->out[l];
   }
-  DecodeSparseArgs sp;
-  sp.q = io->q[sl]; sp.k = io->k[sl]; sp.v = io->v[sl]; sp.wq = io->wq[sl]; sp.wk = io->wk[sl];
-  sp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  sp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
-  sp.kbar = kbar;
-  sp.ksum = ksum;
-  sp.qhat = reinterpret_cast<float*>(ws + w.qhat);
-  sp.counters = reinterpret_cast<unsigned*>(ws + w.counters);
-  // 1. linear layers + sparse prep
-  const RopeFreq rf = rope_freq(D, L.rope_base);
-  const int n_lin = d->n_linear * L.batch * L.heads * (D / 64);
-  const int n_sp = (S.kv_heads + S.q_heads + kDecodeRowsPerCta - 1) / kDecodeRowsPerCta;
-  decode_stage1_kernel<T, D><<<n_lin + S.batch * n_sp, 256, 0, st>>>(
-      a, sp, n_lin, n_sp, L.batch, L.heads, S.q_heads, S.kv_heads, d->cache_capacity, cur_len,
-      S.block, rf, L.rms_eps, S.rms_eps, L.scale);
-  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  // 2. selection
-  const long long capb = d->cache_capacity / S.block;
-  const int width = S.topk + S.n_init + S.n_local;
-  const int bcur = (int)(cur_len / S.block);
-  const int n_cand = std::max(0, bcur - S.n_local + 1 - S.n_init);
-  const int k = std::min(S.topk, n_cand);
-  int chunk = 512, n_chunks = 1;
-  if (k > 0 && k < n_cand) decode_chunks(n_cand, k, &chunk, &n_chunks);
-  const size_t sel_smem = (size_t)std::max(2 * chunk, 2 * n_chunks * k + k) * 4;
-  int32_t* idx = reinterpret_cast<int32_t*>(ws + w.idx);
-  if (allow_smem(decode_select_kernel<D>, sel_smem) != cudaSuccess) return SALA_ERR_CUDA;
-  decode_select_kernel<D><<<S.batch * S.kv_heads * n_chunks, kSelectThreads, sel_smem, st>>>(
-      sp.qhat, kbar, reinterpret_cast<uint32_t*>(ws + w.cand_key),
-      reinterpret_cast<int32_t*>(ws + w.cand_idx), idx, sp.counters, S.q_heads, S.kv_heads, capb, bcur,
-      S.topk, S.n_init, S.n_local, width, chunk, n_chunks);
-  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  // 3. attention partials
+  p.n_linear = d->n_linear;
+  p.B = L.batch;
+  p.H = L.heads;
+  p.eps_l = L.rms_eps;
+  p.scale_l = L.scale;
+  const int sl = d->n_linear;
+  p.q = io->q[sl]; p.k = io->k[sl]; p.v = io->v[sl]; p.gate = io->gate[sl]; p.out = io->out[sl];
+  p.wq = io->wq[sl]; p.wk = io->wk[sl];
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.kbar = kbar;
+  p.ksum = ksum;
+  p.Hq = S.q_heads; p.Hkv = S.kv_heads; p.BLK = S.block; p.topk = S.topk; p.n_init = S.n_init;
+  p.n_local = S.n_local; p.width = S.topk + S.n_init + S.n_local;
+  p.cap = d->cache_capacity;
+  p.capb = d->cache_capacity / S.block;
+  p.pos = cur_len;
+  p.eps_s = S.rms_eps;
+  p.sl2 = sparse_scale(&S) * 1.4426950408889634f;
+  p.bcur = (int)(cur_len / S.block);
+  p.n_cand = std::max(0, p.bcur - S.n_local + 1 - S.n_init);
+  p.kk = std::min(S.topk, p.n_cand);
+  p.n_chunks = std::max(1, (p.n_cand + kDecChunk - 1) / kDecChunk);
+  p.ctl = reinterpret_cast<unsigned*>(ws + w.ctl);
+  p.hist = reinterpret_cast<unsigned*>(ws + w.hist);
+  p.thr = reinterpret_cast<unsigned*>(ws + w.thr);
+  p.keys = reinterpret_cast<uint32_t*>(ws + w.keys);
+  p.above = reinterpret_cast<int*>(ws + w.above);
+  p.bnd = reinterpret_cast<uint2*>(ws + w.bnd);
+  p.idx = reinterpret_cast<int*>(ws + w.idx);
+  p.qhat = reinterpret_cast<float*>(ws + w.qhat);
+  p.part = reinterpret_cast<float*>(ws + w.part);
+  p.rf = rope_freq(D, L.rope_base);
+  // barrier counters, per-(batch, kv head) counts and histograms start at zero
+  if (cudaMemsetAsync(ws, 0, w.zero_bytes, st) != cudaSuccess) return SALA_ERR_CUDA;
   const int G = S.q_heads / S.kv_heads;
-  const int n_parts = (width + kDecodeBlocksPerCta - 1) / kDecodeBlocksPerCta;
-  // K, V staging + queries + logits + running outputs + (m, l) + factors
-  const size_t att_smem = (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
-                          (size_t)G * D * 4 + (size_t)G * 12;
-  if (allow_smem(decode_attn_kernel<T, D>, att_smem) != cudaSuccess) return SALA_ERR_CUDA;
-  float* part = reinterpret_cast<float*>(ws + w.part);
-  decode_attn_kernel<T, D><<<S.batch * S.kv_heads * n_parts, 256, att_smem, st>>>(
-      sp.qhat, sp.k_cache, sp.v_cache, idx, part, S.q_heads, S.kv_heads, d->cache_capacity,
-      cur_len, S.block, width, n_parts, sparse_scale(&S) * 1.4426950408889634f);
-  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  // 4. combine and gate, one CTA per q head
-  const size_t cmb_smem = (size_t)2 * n_parts * 4;
-  if (allow_smem(decode_combine_kernel<T, D>, cmb_smem) != cudaSuccess) return SALA_ERR_CUDA;
-  decode_combine_kernel<T, D><<<S.batch * S.q_heads, D, cmb_smem, st>>>(
-      part, static_cast<const T*>(io->gate[sl]), static_cast<T*>(io->out[sl]), S.q_heads,
-      S.kv_heads, n_parts);
-  return launch_status();
+  const size_t smem = decode_smem_bytes(D, G, S.topk, p.capb, p.width);
+  auto kern = decode_step_kernel<T, D>;
+  if (allow_smem(kern, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) !=
+          cudaSuccess || per_sm < 1)
+    return SALA_ERR_CUDA;
+  const int grid = device_sms() * std::min(per_sm, 1);
+  if (grid < 1) return SALA_ERR_CUDA;
+  void* args[] = {&p};
+  const cudaError_t e = cudaLaunchCooperativeKernel((const void*)kern, grid, kDecThreads, args,
+                                                    smem, st);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e == cudaSuccess ? SALA_OK : SALA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -581,11 +582,11 @@ sala_status sala_decode_step(const sala_decode_desc* d, const sala_decode_io* io
   const int dl = d->lin.head_dim, ds = d->sp.head_dim;
   if (dl != ds) return SALA_ERR_UNSUPPORTED;
   if (d->lin.dtype == SALA_BF16) {
-    if (dl == 128) return run_decode<__nv_bfloat16, 128, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
-    return run_decode<__nv_bfloat16, 64, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+    if (dl == 128) return run_decode<__nv_bfloat16, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+    return run_decode<__nv_bfloat16, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
   }
-  if (dl == 128) return run_decode<float, 128, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
-  return run_decode<float, 64, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+  if (dl == 128) return run_decode<float, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+  return run_decode<float, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
 }
 
 const char* sala_status_string(sala_status s) {

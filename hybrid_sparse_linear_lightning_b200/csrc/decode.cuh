@@ -1,5 +1,5 @@
 // Decode step: one new token through n_linear linear layers and one sparse
-// layer.
+// layer, in ONE cooperative launch.
 //
 // Linear layers keep a constant-size state (MiniCPM-SALA paper, section 2.1):
 //   S <- lam S + k^T v,   o = scale * q^ S,   out = sigmoid(g) * o
@@ -11,11 +11,31 @@
 // initial and local blocks (the block holding the token is local), and runs
 // exact softmax attention over them (split over blocks, then combined).
 //
-// Four launches per token: (1) linear-layer state updates and the sparse
-// layer's normalisation / cache append in one grid; (2) block scores with a
-// per-chunk top-k, merged exactly by the last CTA of each kv head; (3) one
-// CTA per selected block computing partial softmax sums; (4) their combine
-// and the gate, one CTA per q head.
+// The step is bound by HBM traffic (the linear states and the block-mean
+// table) and by the latency of its dependent phases, so it runs as one
+// persistent grid of one CTA per SM whose phases are separated by bounded
+// grid barriers (the launch is cooperative, so every CTA is resident):
+//
+//   P0  every linear (layer, batch, head) state update and output; the
+//       sparse layer's cache append and query normalisation; the scores of
+//       all candidate blocks in chunks of 256, each score also counted in a
+//       4096-bin histogram of its top 12 key bits per (batch, kv head).
+//   B1  the last CTA to arrive finds, per (batch, kv head), the bin T that
+//       holds the k-th largest score.
+//   P1  each chunk emits its candidates above bin T (certainly selected) and
+//       those in bin T (the boundary); the last chunk of a (batch, kv head)
+//       picks the remaining ones from the boundary exactly (score
+//       descending, ties to the lower block) and writes the ascending index
+//       list.  A boundary larger than 1024 entries (degenerate score
+//       distributions) falls back to an exact radix select over all scores.
+//   B2  barrier.
+//   P2  one unit per (batch, kv head, selected block): partial softmax sums
+//       of the group's q heads over that block's keys.
+//   B3  barrier.
+//   P3  one unit per (batch, q head): combine of the partials, output gate.
+//
+// Every wait is bounded (about a second); a barrier that runs out sets the
+// timeout bit of the status word and the CTAs return.
 #pragma once
 
 #include "common.cuh"
@@ -24,32 +44,63 @@
 
 namespace sala {
 
-struct DecodeLinearArgs {
-  const void* q[8];
-  const void* k[8];
-  const void* v[8];
-  const void* gate[8];
-  const float* wq[8];
-  const float* wk[8];
-  const float* lambda[8];
-  float* state[8];
-  void* out[8];
-};
+constexpr int kDecThreads = 512;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecChunk = 256;          // candidate blocks per scoring unit (two threads each)
+constexpr int kDecBinBits = 12;
+constexpr int kDecBins = 1 << kDecBinBits;
+constexpr int kDecBndMax = 1024;        // boundary entries resolved by rank counting
+constexpr int kDecodeMaxQHeads = 64;    // largest sparse-layer q head count the step takes
+constexpr int kDecMaxLayers = 8;
 
-struct DecodeSparseArgs {
+// Control words at the start of the workspace (zeroed by the host before
+// each launch): barrier arrival counts, barrier release flags, and per
+// (batch, kv head) the above / boundary counts and the finished chunks.
+constexpr int kDecCtlBarriers = 4;
+__host__ __device__ constexpr int dec_ctl_words(int bg) { return 2 * kDecCtlBarriers + 4 * bg; }
+
+struct DecodeParams {
+  // linear layers
+  const void* lq[kDecMaxLayers];
+  const void* lk[kDecMaxLayers];
+  const void* lv[kDecMaxLayers];
+  const void* lgate[kDecMaxLayers];
+  const float* lwq[kDecMaxLayers];
+  const float* lwk[kDecMaxLayers];
+  const float* llam[kDecMaxLayers];
+  float* lstate[kDecMaxLayers];
+  void* lout[kDecMaxLayers];
+  int n_linear, B, H;
+  float eps_l, scale_l;
+  // sparse layer
   const void* q;
   const void* k;
   const void* v;
+  const void* gate;
+  void* out;
   const float* wq;
   const float* wk;
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   float* kbar;
   float* ksum;
-  float* qhat;          // [B, Hq, D] normalised queries
-  unsigned* counters;   // [B, Hkv, 2]: selection completion counts (second unused)
+  int Hq, Hkv, BLK, topk, n_init, n_local, width;
+  long long cap, capb, pos;
+  float eps_s, sl2;
+  // selection shape of this step (the same for every batch and kv head)
+  int bcur, n_cand, kk, n_chunks;
+  // workspace
+  unsigned* ctl;
+  unsigned* hist;       // [B * Hkv][kDecBins]
+  unsigned* thr;        // [B * Hkv]
+  uint32_t* keys;       // [B * Hkv][capb]
+  int* above;           // [B * Hkv][topk]
+  uint2* bnd;           // [B * Hkv][kDecBndMax] (key, candidate)
+  int* idx;             // [B * Hkv][width]
+  float* qhat;          // [B][Hq][D]
+  float* part;          // [B * Hkv][width][G][D + 4]
+  RopeFreq rf;
 };
-
 
 // cos / sin of p * base^(-2i/D): the argument is formed and reduced modulo
 // 2 pi in fp64 (|p| < 2^53), then evaluated in fp32 on [-pi, pi].
@@ -60,438 +111,593 @@ __device__ __forceinline__ void rope_cs(long long p, double inv_freq, float& c, 
   sincosf((float)r, &s, &c);
 }
 
-// Stage 1.  CTAs [0, n_lin): one per (linear layer, batch, head, 64-column
-// slice) updating S <- lam S + k^T v and writing out = sigmoid(g) q^ S.
-// CTAs [n_lin, n_lin + B * n_sp): the sparse layer, one warp per row of the
-// Hkv keys and Hq queries of batch b (normalise k and append it and v to the
-// caches, update the running block sum / mean; normalise q); the first of
-// them also resets the completion counters.
-constexpr int kDecodeMaxQHeads = 64;   // largest sparse-layer q head count the decode step takes
-constexpr int kDecodeRowsPerCta = 8;   // sparse-layer rows per stage-1 CTA
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
-template <typename T, int D>
-__global__ void __launch_bounds__(256)
-decode_stage1_kernel(DecodeLinearArgs a, DecodeSparseArgs sp, int n_lin, int n_sp, int B, int H,
-                     int Hq, int Hkv, long long cap, long long pos, int BLK, RopeFreq rf,
-                     float eps_l, float eps_s, float scale) {
-  __shared__ float sh[D * 3 + 256];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if ((int)blockIdx.x < n_lin) {
-    constexpr int NSL = D / 64;
-    float* qh = sh;
-    float* kh = sh + D;
-    float* vv = sh + 2 * D;
-    float* part = sh + 3 * D;          // [4][64]
-    const int slice = blockIdx.x % NSL;
-    const int h = (blockIdx.x / NSL) % H;
-    const int b = (blockIdx.x / (NSL * H)) % B;
-    const int layer = blockIdx.x / (NSL * H * B);
-    const long long voff = ((long long)b * H + h) * D;
-    if (warp < 2) {
-      const T* src = static_cast<const T*>(warp == 0 ? a.q[layer] : a.k[layer]);
-      const float* w = warp == 0 ? a.wq[layer] : a.wk[layer];
-      float* dst = warp == 0 ? qh : kh;
-      float ss = 0.f;
-      for (int e = lane; e < D; e += 32) { const float x = to_f32(src[voff + e]); ss += x * x; }
-      ss = warp_sum(ss);
-      const float r = rsqrtf(ss / D + eps_l);
-      for (int i = lane; i < D / 2; i += 32) {
-        const float x1 = to_f32(src[voff + i]) * r * w[i];
-        const float x2 = to_f32(src[voff + i + D / 2]) * r * w[i + D / 2];
-        float c, s;
-        rope_cs(pos, rf.inv[i], c, s);
-        dst[i] = x1 * c - x2 * s;
-        dst[i + D / 2] = x2 * c + x1 * s;
-      }
-    } else if (warp == 2) {
-      const T* v = static_cast<const T*>(a.v[layer]);
-      for (int e = lane; e < D; e += 32) vv[e] = to_f32(v[voff + e]);
-    }
-    __syncthreads();
-    const int col = slice * 64 + (tid & 63);
-    const int rg = tid >> 6;
-    const float lam = a.lambda[layer][h];
-    float* S = a.state[layer] + ((long long)b * H + h) * D * D;
-    const float vc = vv[col];
-    // all D/4 state loads of this thread are in flight before the first use
-    constexpr int RPT = D / 4;
-    float sv[RPT];
-#pragma unroll
-    for (int u = 0; u < RPT; ++u) sv[u] = S[(long long)(rg * RPT + u) * D + col];
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int u = 0; u < RPT; u += 2) {
-      const int r = rg * RPT + u;
-      const float s0 = lam * sv[u] + kh[r] * vc;
-      const float s1 = lam * sv[u + 1] + kh[r + 1] * vc;
-      S[(long long)r * D + col] = s0;
-      S[(long long)(r + 1) * D + col] = s1;
-      acc0 = fmaf(qh[r], s0, acc0);
-      acc1 = fmaf(qh[r + 1], s1, acc1);
-    }
-    part[rg * 64 + (tid & 63)] = acc0 + acc1;
-    __syncthreads();
-    if (tid < 64) {
-      const float o = scale * (part[tid] + part[64 + tid] + part[128 + tid] + part[192 + tid]);
-      const T* g = static_cast<const T*>(a.gate[layer]);
-      T* out = static_cast<T*>(a.out[layer]);
-      out[voff + col] = from_f32<T>(sigmoidf_(to_f32(g[voff + col])) * o);
-    }
-    return;
+// Grid barrier of a cooperative launch, bounded like every wait here.  The
+// last CTA to arrive runs `last` (whole CTA) before releasing the others.
+// Returns false (and sets the timeout bit) if the release did not come.
+template <typename F>
+__device__ __forceinline__ bool dec_grid_sync(unsigned* count, unsigned* flag, F last) {
+  __shared__ int s_last, s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(count, 1u) == gridDim.x - 1;
   }
-  // ---- sparse layer of batch b, rows [rc * 8, rc * 8 + 8) of its Hkv + Hq
-  const int b = (blockIdx.x - n_lin) / n_sp;
-  const int rc = (blockIdx.x - n_lin) % n_sp;
-  const bool closes = ((pos + 1) % BLK) == 0;
-  const T* q = static_cast<const T*>(sp.q);
-  const T* k = static_cast<const T*>(sp.k);
-  const T* v = static_cast<const T*>(sp.v);
-  if (rc == 0 && tid < 2 * Hkv) sp.counters[(long long)b * Hkv * 2 + tid] = 0u;
-  {
-    const int r = rc * kDecodeRowsPerCta + warp;
-    if (warp >= kDecodeRowsPerCta || r >= Hkv + Hq) return;
-    const bool isk = r < Hkv;
-    const int h = isk ? r : r - Hkv;
-    const T* src = isk ? k + ((long long)b * Hkv + h) * D : q + ((long long)b * Hq + h) * D;
-    const float* w = isk ? sp.wk : sp.wq;
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    last();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      atomicExch(flag, 1u);
+      s_ok = 1;
+    }
+  } else if (threadIdx.x == 0) {
+    s_ok = 1;
+    if (ld_acquire_u32(flag) == 0u) {
+      const long long t0 = clock64();
+      while (ld_acquire_u32(flag) == 0u) {
+        if (clock64() - t0 > (1ll << 31)) {
+          set_status(kStatusTimeout);
+          s_ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+template <typename T>
+__device__ __forceinline__ float ldf(const void* p, long long i) {
+  return to_f32(static_cast<const T*>(p)[i]);
+}
+
+// ------------------------------------------------------------------ P0 units
+
+// Normalised query of q head h of batch b (RMSNorm over D, no rotation):
+// one warp, D/32 values per lane.
+template <typename T, int D>
+__device__ __forceinline__ void norm_query_warp(const DecodeParams& p, int b, int h, float* x) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) {
+    x[e] = ldf<T>(p.q, ((long long)b * p.Hq + h) * D + lane + 32 * e);
+    ss += x[e] * x[e];
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / D + p.eps_s);
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) x[e] = x[e] * r * p.wq[lane + 32 * e];
+}
+
+// Scores of candidate blocks [c0, c0 + nc) of (b, g) against the group's
+// summed normalised query; each score's key goes to `keys` and to the
+// (b, g) histogram.
+template <typename T, int D>
+__device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
+  const int ck = u % p.n_chunks;
+  const int bg = u / p.n_chunks;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* qh = sm;              // [kDecWarps][D] per-warp partial group sums
+  float* qv = sm + kDecWarps * D;
+  // this thread's half row of its candidate's block mean is loaded first, so
+  // that the loads are in flight while the group query is formed
+  const int c0 = ck * kDecChunk;
+  const int nc = min(kDecChunk, p.n_cand - c0);
+  const int c = tid >> 1, half = tid & 1;
+  float4 kv[D / 8];
+  if (c < nc) {
+    const float4* kr = reinterpret_cast<const float4*>(
+        p.kbar + (((long long)b * p.capb + p.n_init + c0 + c) * p.Hkv + g) * D + half * (D / 2));
+#pragma unroll
+    for (int e = 0; e < D / 8; ++e) kv[e] = kr[e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < D / 8; ++e) kv[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float acc[D / 32];
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+  for (int h = warp; h < G; h += kDecWarps) {
     float x[D / 32];
+    norm_query_warp<T, D>(p, b, g * G + h, x);
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) acc[e] += x[e];
+  }
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) qh[warp * D + lane + 32 * e] = acc[e];
+  __syncthreads();
+  if (tid < D) {
+    float s = 0.f;
+    for (int w = 0; w < kDecWarps; ++w) s += qh[w * D + tid];
+    qv[tid] = s;
+  }
+  __syncthreads();
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  {
+    const float* qq = qv + half * (D / 2);
+#pragma unroll
+    for (int e = 0; e < D / 8; ++e) {
+      s0 = fmaf(qq[4 * e], kv[e].x, s0);
+      s1 = fmaf(qq[4 * e + 1], kv[e].y, s1);
+      s2 = fmaf(qq[4 * e + 2], kv[e].z, s2);
+      s3 = fmaf(qq[4 * e + 3], kv[e].w, s3);
+    }
+  }
+  float s = (s0 + s1) + (s2 + s3);
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  if (c < nc && half == 0) {
+    const uint32_t key = score_key(s * rsqrtf((float)D));
+    p.keys[(long long)bg * p.capb + c0 + c] = key;
+    atomicAdd(p.hist + (long long)bg * kDecBins + (key >> (32 - kDecBinBits)), 1u);
+  }
+}
+
+// One linear (layer, batch, head): S <- lam S + k^T v over the whole d x d
+// state, out = sigmoid(g) * scale * q^ S.  Thread (row group rg of 32 rows,
+// column col).
+template <typename T, int D>
+__device__ void dec_linear_unit(const DecodeParams& p, int u, float* sm) {
+  const int h = u % p.H;
+  const int b = (u / p.H) % p.B;
+  const int layer = u / (p.H * p.B);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* qh = sm;
+  float* kh = sm + D;
+  float* vv = sm + 2 * D;
+  float* part = sm + 3 * D;          // [4][D]
+  const long long voff = ((long long)b * p.H + h) * D;
+  const int col = tid & (D - 1);
+  const int rg = tid / D;                       // D = 128: four groups of 32 rows; D = 64: eight of 8
+  constexpr int NRG = kDecThreads / D;
+  constexpr int RPT = D / NRG;
+  float* S = p.lstate[layer] + ((long long)b * p.H + h) * D * D;
+  // the state loads are issued before the token's norm and rotation
+  float sv[RPT];
+#pragma unroll
+  for (int u2 = 0; u2 < RPT; ++u2) sv[u2] = S[(long long)(rg * RPT + u2) * D + col];
+  if (warp < 2) {
+    const void* src = warp == 0 ? p.lq[layer] : p.lk[layer];
+    const float* w = warp == 0 ? p.lwq[layer] : p.lwk[layer];
+    float* dst = warp == 0 ? qh : kh;
     float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < D / 32; ++e) { x[e] = to_f32(src[lane + 32 * e]); ss += x[e] * x[e]; }
+    for (int e = lane; e < D; e += 32) { const float x = ldf<T>(src, voff + e); ss += x * x; }
     ss = warp_sum(ss);
-    const float rn = rsqrtf(ss / D + eps_s);
+    const float r = rsqrtf(ss / D + p.eps_l);
+    for (int i = lane; i < D / 2; i += 32) {
+      const float x1 = ldf<T>(src, voff + i) * r * w[i];
+      const float x2 = ldf<T>(src, voff + i + D / 2) * r * w[i + D / 2];
+      float c, s;
+      rope_cs(p.pos, p.rf.inv[i], c, s);
+      dst[i] = x1 * c - x2 * s;
+      dst[i + D / 2] = x2 * c + x1 * s;
+    }
+  } else if (warp == 2) {
+    for (int e = lane; e < D; e += 32) vv[e] = ldf<T>(p.lv[layer], voff + e);
+  }
+  __syncthreads();
+  const float lam = p.llam[layer][h];
+  const float vc = vv[col];
+  float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) x[e] = x[e] * rn * w[lane + 32 * e];
-    if (isk) {
-      const long long crow = (((long long)b * cap + pos) * Hkv + h) * D;
-      float* ks = sp.ksum + ((long long)b * Hkv + h) * D;
+  for (int u2 = 0; u2 < RPT; u2 += 2) {
+    const int r = rg * RPT + u2;
+    const float s0 = lam * sv[u2] + kh[r] * vc;
+    const float s1 = lam * sv[u2 + 1] + kh[r + 1] * vc;
+    S[(long long)r * D + col] = s0;
+    S[(long long)(r + 1) * D + col] = s1;
+    acc0 = fmaf(qh[r], s0, acc0);
+    acc1 = fmaf(qh[r + 1], s1, acc1);
+  }
+  part[rg * D + col] = acc0 + acc1;
+  __syncthreads();
+  if (tid < D) {
+    float o = 0.f;
+#pragma unroll
+    for (int r = 0; r < NRG; ++r) o += part[r * D + tid];
+    o *= p.scale_l;
+    T* out = static_cast<T*>(p.lout[layer]);
+    out[voff + tid] = from_f32<T>(sigmoidf_(ldf<T>(p.lgate[layer], voff + tid)) * o);
+  }
+}
+
+// The sparse layer's new token of batch b: normalise its key (append key and
+// value to the caches, add to the running block sum, close the block mean
+// when the block completes) and its queries (kept in fp32 for P2).  One warp
+// per row.
+template <typename T, int D>
+__device__ void dec_sparse_prep_unit(const DecodeParams& p, int b) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool closes = ((p.pos + 1) % p.BLK) == 0;
+  for (int r = warp; r < p.Hkv + p.Hq; r += kDecWarps) {
+    float x[D / 32];
+    if (r < p.Hkv) {
+      const int h = r;
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < D / 32; ++e) {
+        x[e] = ldf<T>(p.k, ((long long)b * p.Hkv + h) * D + lane + 32 * e);
+        ss += x[e] * x[e];
+      }
+      ss = warp_sum(ss);
+      const float rn = rsqrtf(ss / D + p.eps_s);
+      const long long crow = (((long long)b * p.cap + p.pos) * p.Hkv + h) * D;
+      float* ks = p.ksum + ((long long)b * p.Hkv + h) * D;
 #pragma unroll
       for (int e = 0; e < D / 32; ++e) {
         const int d = lane + 32 * e;
-        sp.k_cache[crow + d] = __float2bfloat16_rn(x[e]);
-        sp.v_cache[crow + d] = __float2bfloat16_rn(to_f32(v[((long long)b * Hkv + h) * D + d]));
-        const float s = ks[d] + x[e];
+        const float xn = x[e] * rn * p.wk[d];
+        p.k_cache[crow + d] = __float2bfloat16_rn(xn);
+        p.v_cache[crow + d] = __float2bfloat16_rn(ldf<T>(p.v, ((long long)b * p.Hkv + h) * D + d));
+        const float s = ks[d] + xn;
         if (closes) {
-          sp.kbar[(((long long)b * (cap / BLK) + pos / BLK) * Hkv + h) * D + d] = s / (float)BLK;
+          p.kbar[(((long long)b * p.capb + p.pos / p.BLK) * p.Hkv + h) * D + d] = s / (float)p.BLK;
           ks[d] = 0.f;
         } else {
           ks[d] = s;
         }
       }
     } else {
+      const int h = r - p.Hkv;
+      norm_query_warp<T, D>(p, b, h, x);
 #pragma unroll
-      for (int e = 0; e < D / 32; ++e) sp.qhat[((long long)b * Hq + h) * D + lane + 32 * e] = x[e];
+      for (int e = 0; e < D / 32; ++e) p.qhat[((long long)b * p.Hq + h) * D + lane + 32 * e] = x[e];
     }
   }
 }
 
-// Top-k of the scored candidates: rows of the candidate chunks and, in the
-// last CTA of each (batch, kv head), the exact merge.  Chunk `ck` scores
-// candidates [ck * chunk, ck * chunk + chunk) of [n_init, n_init + n_cand)
-// and keeps its local top-k (ascending block order); the union of the local
-// lists contains the global top-k, so the last CTA selects it exactly (same
-// tie rule: equal scores go to the lower block).  Dynamic smem: chunk keys.
+// ------------------------------------------------------------------ B1, P1
+
+// Bin of the k-th largest key of every (batch, kv head): the last CTA at the
+// first barrier scans each 4096-bin histogram from the top.  Thread t owns
+// the 8 bins 4095 - 8t - u, u = 0..7.
+__device__ void dec_find_thresholds(const DecodeParams& p, int* scratch) {
+  static_assert(kDecBins == 8 * kDecThreads, "eight bins per thread");
+  const int tid = threadIdx.x;
+  for (int bg = 0; bg < p.B * p.Hkv; ++bg) {
+    const unsigned* h = p.hist + (long long)bg * kDecBins;
+    int cnt[8], tot = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) { cnt[u] = (int)__ldcg(h + kDecBins - 1 - 8 * tid - u); tot += cnt[u]; }
+    int all;
+    const int before = block_exclusive_scan<kDecThreads>(tot, scratch, &all);
+    if (before < p.kk && before + tot >= p.kk) {
+      int cum = before, u = 0;
+      for (; u < 8; ++u) {
+        if (cum + cnt[u] >= p.kk) break;
+        cum += cnt[u];
+      }
+      p.thr[bg] = (unsigned)(kDecBins - 1 - 8 * tid - u);
+    }
+    __syncthreads();
+  }
+}
+
+// Exact choice of the selected candidates of (b, g) once every chunk has
+// emitted: the `above` list plus the best (kk - n_above) boundary entries by
+// (key descending, candidate ascending), written as the ascending index row.
 template <int D>
-__global__ void __launch_bounds__(kSelectThreads)
-decode_select_kernel(const float* __restrict__ qhat, const float* __restrict__ kbar,
-                     uint32_t* __restrict__ cand_key, int32_t* __restrict__ cand_idx,
-                     int32_t* __restrict__ idx, unsigned* __restrict__ counters, int Hq, int Hkv,
-                     long long cap_blocks, int bcur, int topk, int n_init, int n_local, int width,
-                     int chunk, int n_chunks) {
-  extern __shared__ uint32_t keys[];        // max(chunk, n_chunks * k) keys + as many ints
-  __shared__ float qv[D];
-  __shared__ int hist[256];
-  __shared__ int scan_scratch[kSelectThreads / 32 + 1];
+__device__ void dec_resolve(const DecodeParams& p, int bg, unsigned char* smem_raw) {
+  const int tid = threadIdx.x;
+  unsigned* ctl = p.ctl + 2 * kDecCtlBarriers + 4 * bg;
+  const int n_above = (int)min(ld_acquire_u32(ctl + 0), (unsigned)p.topk);
+  const int n_bnd = (int)ld_acquire_u32(ctl + 1);
+  const int need = p.kk - n_above;
+  int32_t* chosen = reinterpret_cast<int32_t*>(smem_raw);          // [topk]
+  int32_t* sorted = chosen + p.topk;                               // [topk]
+  uint8_t* tail = reinterpret_cast<uint8_t*>(sorted + p.topk);
+  tail = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tail) + 15) & ~uintptr_t(15));
+  __shared__ int hist_s[256];
+  __shared__ int scan_s[kDecThreads / 32 + 1];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
-  __shared__ int s_last;
-  const int ck = blockIdx.x % n_chunks;
-  const int g = (blockIdx.x / n_chunks) % Hkv;
-  const int b = blockIdx.x / (n_chunks * Hkv);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int32_t* row = idx + ((long long)b * Hkv + g) * width;
-  const int n_cand = max(0, bcur - n_local + 1 - n_init);
-  const int k = min(topk, n_cand);
-  const int n_first = min(n_init, bcur + 1);
-  const int local_lo = max(n_init, bcur - n_local + 1);
-  const int n_loc = max(0, bcur - local_lo + 1);
-  if (k == 0 || k == n_cand) {
-    if (ck != 0) return;
-    for (int e = tid; e < n_first; e += kSelectThreads) row[e] = e;
-    for (int e = tid; e < k; e += kSelectThreads) row[n_first + e] = n_init + e;
-    for (int e = tid; e < n_loc; e += kSelectThreads) row[n_first + k + e] = local_lo + e;
-    for (int e = n_first + k + n_loc + tid; e < width; e += kSelectThreads) row[e] = -1;
-    return;
-  }
-  // ---- score this chunk
-  const int c0 = ck * chunk, nc = min(chunk, n_cand - c0);
-  // group-summed query (fixed head order)
-  const int G = Hq / Hkv;
-  for (int e = tid; e < D; e += kSelectThreads) {
-    float s = 0.f;
-    for (int hh = 0; hh < G; ++hh) s += qhat[((long long)b * Hq + g * G + hh) * D + e];
-    qv[e] = s;
-  }
-  __syncthreads();
-  // one thread per candidate: its whole block-mean row is read with 16-byte
-  // loads that are all independent, so many rows are in flight at once
-  const float inv_sqrt_d = rsqrtf((float)D);
-  for (int c = tid; c < nc; c += kSelectThreads) {
-    const float4* kr = reinterpret_cast<const float4*>(
-        kbar + (((long long)b * cap_blocks + n_init + c0 + c) * Hkv + g) * D);
-    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-    for (int e = 0; e < D / 4; ++e) {
-      const float4 kv = kr[e];
-      p0 = fmaf(qv[4 * e], kv.x, p0);
-      p1 = fmaf(qv[4 * e + 1], kv.y, p1);
-      p2 = fmaf(qv[4 * e + 2], kv.z, p2);
-      p3 = fmaf(qv[4 * e + 3], kv.w, p3);
+  bool in_order = false;
+  if (n_bnd <= kDecBndMax && need >= 1 && need <= n_bnd) {
+    uint2* sb = reinterpret_cast<uint2*>(tail);
+    for (int e = tid; e < n_above; e += kDecThreads) chosen[e] = __ldcg(p.above + (long long)bg * p.topk + e);
+    for (int e = tid; e < n_bnd; e += kDecThreads) sb[e] = __ldcg(p.bnd + (long long)bg * kDecBndMax + e);
+    __syncthreads();
+    for (int e = tid; e < n_bnd; e += kDecThreads) {
+      const uint2 me = sb[e];
+      int rank = 0;
+      for (int f = 0; f < n_bnd; ++f) {
+        const uint2 o = sb[f];
+        rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+      }
+      if (rank < need) chosen[n_above + rank] = (int)me.y;
     }
-    keys[c] = score_key(((p0 + p1) + (p2 + p3)) * inv_sqrt_d);
-  }
-  (void)lane;
-  (void)warp;
-  __syncthreads();
-  // ---- local top-k: positions into the ints after the keys
-  int32_t* pos_list = reinterpret_cast<int32_t*>(keys + chunk);
-  const int kl = min(k, nc);
-  if (kl == nc) {
-    for (int e = tid; e < nc; e += kSelectThreads) pos_list[e] = e;
   } else {
-    topk_emit_sorted(keys, nc, kl, pos_list, 0, hist, scan_scratch, &s_prefix, &s_need);
+    // degenerate boundary: exact radix select over every score of (b, g)
+    uint32_t* sk = reinterpret_cast<uint32_t*>(tail);
+    for (int e = tid; e < p.n_cand; e += kDecThreads) sk[e] = __ldcg(p.keys + (long long)bg * p.capb + e);
+    __syncthreads();
+    topk_emit_sorted<kDecThreads>(sk, p.n_cand, p.kk, sorted, 0, hist_s, scan_s, &s_prefix,
+                                  &s_need);
+    in_order = true;
   }
   __syncthreads();
-  const long long cbase = (((long long)b * Hkv + g) * n_chunks + ck) * topk;
-  for (int e = tid; e < k; e += kSelectThreads) {
-    if (e < kl) {
-      cand_key[cbase + e] = keys[pos_list[e]];
-      cand_idx[cbase + e] = n_init + c0 + pos_list[e];
-    } else {
-      cand_key[cbase + e] = 0u;       // below every real score key
-      cand_idx[cbase + e] = -1;
+  if (!in_order) {
+    for (int e = tid; e < p.kk; e += kDecThreads) {
+      const int me = chosen[e];
+      int r = 0;
+      for (int f = 0; f < p.kk; ++f) r += chosen[f] < me;
+      sorted[r] = me;
     }
+    __syncthreads();
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0)
-    s_last = atomicAdd(counters + ((long long)b * Hkv + g) * 2, 1u) == (unsigned)(n_chunks - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // ---- exact merge of the n_chunks local lists (chunk order = block order)
-  const int total = n_chunks * k;
-  uint32_t* mk = keys;
-  int32_t* mi = reinterpret_cast<int32_t*>(keys + total);
-  const long long gbase = ((long long)b * Hkv + g) * n_chunks * topk;
-  for (int e = tid; e < total; e += kSelectThreads) {
-    const int chk = e / k, r = e % k;
-    mk[e] = cand_key[gbase + (long long)chk * topk + r];
-    mi[e] = cand_idx[gbase + (long long)chk * topk + r];
-  }
-  __syncthreads();
-  int32_t* chosen = mi + total;       // k positions
-  topk_emit_sorted(mk, total, k, chosen, 0, hist, scan_scratch, &s_prefix, &s_need);
-  __syncthreads();
-  for (int e = tid; e < n_first; e += kSelectThreads) row[e] = e;
-  for (int e = tid; e < k; e += kSelectThreads) row[n_first + e] = mi[chosen[e]];
-  for (int e = tid; e < n_loc; e += kSelectThreads) row[n_first + k + e] = local_lo + e;
-  for (int e = n_first + k + n_loc + tid; e < width; e += kSelectThreads) row[e] = -1;
+  const int b_ = p.bcur;
+  const int n_first = min(p.n_init, b_ + 1);
+  const int local_lo = max(p.n_init, b_ - p.n_local + 1);
+  const int n_loc = max(0, b_ - local_lo + 1);
+  int32_t* row = p.idx + (long long)bg * p.width;
+  for (int e = tid; e < n_first; e += kDecThreads) row[e] = e;
+  for (int e = tid; e < p.kk; e += kDecThreads) row[n_first + e] = p.n_init + sorted[e];
+  for (int e = tid; e < n_loc; e += kDecThreads) row[n_first + p.kk + e] = local_lo + e;
+  for (int e = n_first + p.kk + n_loc + tid; e < p.width; e += kDecThreads) row[e] = -1;
 }
 
-// Partial attention of the group's G heads over up to kDecodeBlocksPerCta
-// selected blocks (online softmax across them).  Keys / values are staged as
-// bf16 in shared memory with 16-byte chunks XOR-swizzled by row; the next
-// block's loads are in flight while the current one is processed.  Partials:
-// [B, Hkv, n_parts, G, D + 4] = (m, l, -, -, o[D]) in base-2 logits; they are
-// combined by decode_combine_kernel.
-constexpr int kDecodeBlocksPerCta = 1;
+// Index row when no ranking is needed (no candidates, or k covers them all).
+__device__ void dec_direct_row(const DecodeParams& p, int bg) {
+  const int tid = threadIdx.x;
+  const int b_ = p.bcur;
+  const int n_first = min(p.n_init, b_ + 1);
+  const int local_lo = max(p.n_init, b_ - p.n_local + 1);
+  const int n_loc = max(0, b_ - local_lo + 1);
+  int32_t* row = p.idx + (long long)bg * p.width;
+  for (int e = tid; e < n_first; e += kDecThreads) row[e] = e;
+  for (int e = tid; e < p.kk; e += kDecThreads) row[n_first + e] = p.n_init + e;
+  for (int e = tid; e < n_loc; e += kDecThreads) row[n_first + p.kk + e] = local_lo + e;
+  for (int e = n_first + p.kk + n_loc + tid; e < p.width; e += kDecThreads) row[e] = -1;
+}
 
-template <typename T, int D>
-__global__ void __launch_bounds__(256)
-decode_attn_kernel(const float* __restrict__ qhat, const __nv_bfloat16* __restrict__ k_cache,
-                   const __nv_bfloat16* __restrict__ v_cache, const int32_t* __restrict__ idx,
-                   float* __restrict__ part, int Hq, int Hkv, long long cap, long long pos,
-                   int BLK, int width, int n_parts, float sl2) {
-  constexpr int NC = D / 8;                 // 16-byte chunks per row
+template <int D>
+__device__ void dec_emit_unit(const DecodeParams& p, int u, unsigned char* smem_raw) {
+  const int ck = u % p.n_chunks;
+  const int bg = u / p.n_chunks;
+  const int tid = threadIdx.x;
+  unsigned* ctl = p.ctl + 2 * kDecCtlBarriers + 4 * bg;
+  const unsigned T = __ldcg(p.thr + bg);
+  const int c0 = ck * kDecChunk;
+  const int nc = min(kDecChunk, p.n_cand - c0);
+  for (int c = tid; c < nc; c += kDecThreads) {
+    const uint32_t key = __ldcg(p.keys + (long long)bg * p.capb + c0 + c);
+    const unsigned bin = key >> (32 - kDecBinBits);
+    if (bin > T) {
+      const unsigned slot = atomicAdd(ctl + 0, 1u);
+      if (slot < (unsigned)p.topk) p.above[(long long)bg * p.topk + slot] = c0 + c;
+      else set_status(kStatusBounds);
+    } else if (bin == T) {
+      const unsigned slot = atomicAdd(ctl + 1, 1u);
+      if (slot < (unsigned)kDecBndMax) p.bnd[(long long)bg * kDecBndMax + slot] = make_uint2(key, c0 + c);
+    }
+  }
+  __shared__ int s_last_chunk;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last_chunk = atomicAdd(ctl + 2, 1u) == (unsigned)(p.n_chunks - 1);
+  }
+  __syncthreads();
+  if (s_last_chunk) {
+    __threadfence();
+    dec_resolve<D>(p, bg, smem_raw);
+  }
+}
+
+// ------------------------------------------------------------------ P2, P3
+
+// Partial softmax sums of the G q heads of (b, g) over selected block `slot`:
+// [G][D + 4] = (m, l, -, -, o[D]) with logits in base 2.  Keys and values are
+// staged as bf16 with 16-byte chunks XOR-swizzled by row.
+template <int D>
+__device__ void dec_attn_unit(const DecodeParams& p, int u, unsigned char* smem_raw) {
+  constexpr int NC = D / 8;
   constexpr int DP = D + 4;
-  constexpr int PER = 64 * NC / 256;        // 16-byte K (and V) chunks per thread and block
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int slot = u % p.width;
+  const int bg = u / p.width;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint4* ks = reinterpret_cast<uint4*>(smem_raw);                 // [64][NC]
   uint4* vs = ks + 64 * NC;                                       // [64][NC]
-  const int G = Hq / Hkv;
   float* qs = reinterpret_cast<float*>(vs + 64 * NC);             // [G][D]
   float* lg = qs + G * D;                                         // [G][64]
-  float* os = lg + G * 64;                                        // [G][D] running outputs
-  float* ml = os + G * D;                                         // [G][2] running (m, l)
-  float* fs = ml + 2 * G;                                         // [G] rescale factors
-  const int pidx = blockIdx.x % n_parts;
-  const int g = (blockIdx.x / n_parts) % Hkv;
-  const int b = blockIdx.x / (n_parts * Hkv);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int32_t* irow = idx + ((long long)b * Hkv + g) * width;
-  float* pbase = part + (((long long)b * Hkv + g) * n_parts + pidx) * G * DP;
-  const int slot0 = pidx * kDecodeBlocksPerCta;
-  const int nslot = min(kDecodeBlocksPerCta, width - slot0);
-  // blocks of this CTA that hold keys (entries of the list are ascending)
-  auto block_of = [&](int u) -> int {
-    const int j = irow[slot0 + u];
-    if (j >= 0 && (long long)j * BLK > pos) {
-      set_status(kStatusBounds);
-      return -1;
-    }
-    return j;
-  };
-  auto load_block = [&](int j, uint4* kr, uint4* vr) {
-    const long long kend = ((long long)(j + 1) * BLK < pos + 1) ? (long long)(j + 1) * BLK : pos + 1;
-    const int nk = (int)(kend - (long long)j * BLK);
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      const int e = tid + 256 * u, sr = e / NC, c = e % NC;
-      kr[u] = vr[u] = make_uint4(0, 0, 0, 0);
-      if (sr < nk) {
-        const long long off = (((long long)b * cap + (long long)j * BLK + sr) * Hkv + g) * D + 8 * c;
-        kr[u] = *reinterpret_cast<const uint4*>(k_cache + off);
-        vr[u] = *reinterpret_cast<const uint4*>(v_cache + off);
-      }
-    }
-    return nk;
-  };
-  {
-    const float4* qsrc = reinterpret_cast<const float4*>(qhat + ((long long)b * Hq + g * G) * D);
-    float4* qdst = reinterpret_cast<float4*>(qs);
-    for (int e = tid; e < G * D / 4; e += 256) qdst[e] = qsrc[e];
-    for (int e = tid; e < G * D; e += 256) os[e] = 0.f;
-    for (int e = tid; e < G; e += 256) { ml[2 * e] = -INFINITY; ml[2 * e + 1] = 0.f; }
+  float* red = lg + G * 64;                                       // [2][G][D]
+  float* ml = red + 2 * G * D;                                    // [G][2]
+  float* pb = p.part + ((long long)bg * p.width + slot) * G * DP;
+  int j = __ldcg(p.idx + (long long)bg * p.width + slot);
+  if (j >= 0 && (long long)j * p.BLK > p.pos) {
+    set_status(kStatusBounds);
+    j = -1;
   }
-  uint4 kr[PER], vr[PER];
-  int u = 0, j = -1, nk = 0;
-  while (u < nslot && (j = block_of(u)) < 0) ++u;
-  if (j >= 0) nk = load_block(j, kr, vr);
-  while (j >= 0) {
-    __syncthreads();                      // previous block's readers are done
-#pragma unroll
-    for (int w = 0; w < PER; ++w) {
-      const int e = tid + 256 * w, sr = e / NC, c = e % NC;
-      ks[sr * NC + (c ^ (sr & (NC - 1)))] = kr[w];
-      vs[sr * NC + (c ^ (sr & (NC - 1)))] = vr[w];
+  if (j < 0) {
+    for (int e = tid; e < G * DP; e += kDecThreads) pb[e] = (e % DP) == 0 ? -INFINITY : 0.f;
+    return;
+  }
+  const long long kend = min((long long)(j + 1) * p.BLK, p.pos + 1);
+  const int nk = (int)(kend - (long long)j * p.BLK);
+  for (int e = tid; e < 64 * NC; e += kDecThreads) {
+    const int sr = e / NC, c = e % NC;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+    if (sr < nk) {
+      const long long off = (((long long)b * p.cap + (long long)j * p.BLK + sr) * p.Hkv + g) * D + 8 * c;
+      kv = __ldcg(reinterpret_cast<const uint4*>(p.k_cache + off));
+      vv = __ldcg(reinterpret_cast<const uint4*>(p.v_cache + off));
     }
-    const int cur_nk = nk;
-    // next block's loads overlap this block's arithmetic
-    int jn = -1;
-    ++u;
-    while (u < nslot && (jn = block_of(u)) < 0) ++u;
-    if (u >= nslot) jn = -1;
-    if (jn >= 0) nk = load_block(jn, kr, vr);
-    __syncthreads();
-    // logits: thread (key s, head hq + 4 m)
-    {
-      const int sr = tid & 63;
-      for (int h = tid >> 6; h < G; h += 4) {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        const float* qr = qs + h * D;
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          float kf[8];
-          load8(reinterpret_cast<const __nv_bfloat16*>(&ks[sr * NC + (c ^ (sr & (NC - 1)))]), kf);
-          a0 = fmaf(kf[0], qr[8 * c + 0], a0); a1 = fmaf(kf[1], qr[8 * c + 1], a1);
-          a2 = fmaf(kf[2], qr[8 * c + 2], a2); a3 = fmaf(kf[3], qr[8 * c + 3], a3);
-          a0 = fmaf(kf[4], qr[8 * c + 4], a0); a1 = fmaf(kf[5], qr[8 * c + 5], a1);
-          a2 = fmaf(kf[6], qr[8 * c + 6], a2); a3 = fmaf(kf[7], qr[8 * c + 7], a3);
-        }
-        lg[h * 64 + sr] = sr < cur_nk ? ((a0 + a1) + (a2 + a3)) * sl2 : -INFINITY;
-      }
-    }
-    __syncthreads();
-    // online softmax per head (one warp per head, two logits per lane)
-    for (int h = warp; h < G; h += 8) {
-      const float x0 = lg[h * 64 + lane], x1 = lg[h * 64 + lane + 32];
-      const float mo = ml[2 * h];
-      const float mn = fmaxf(mo, warp_max(fmaxf(x0, x1)));
-      const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn);
-      const float ls = warp_sum(p0 + p1);
-      lg[h * 64 + lane] = p0;
-      lg[h * 64 + lane + 32] = p1;
-      if (lane == 0) {
-        const float f = mo == -INFINITY ? 0.f : exp2f(mo - mn);
-        fs[h] = f;
-        ml[2 * h] = mn;
-        ml[2 * h + 1] = ml[2 * h + 1] * f + ls;
-      }
-    }
-    __syncthreads();
-    // O = f O + P V: thread (head, 8-column chunk)
-    for (int e = tid; e < G * NC; e += 256) {
-      const int h = e / NC, c = e % NC;
-      float o[8];
-      const float f = fs[h];
-#pragma unroll
-      for (int w = 0; w < 8; ++w) o[w] = os[h * D + 8 * c + w] * f;
-      for (int sr = 0; sr < cur_nk; ++sr) {
-        float vf[8];
-        load8(reinterpret_cast<const __nv_bfloat16*>(&vs[sr * NC + (c ^ (sr & (NC - 1)))]), vf);
-        const float p = lg[h * 64 + sr];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) o[w] = fmaf(p, vf[w], o[w]);
-      }
-#pragma unroll
-      for (int w = 0; w < 8; ++w) os[h * D + 8 * c + w] = o[w];
-    }
-    j = jn;
+    ks[sr * NC + (c ^ (sr & (NC - 1)))] = kv;
+    vs[sr * NC + (c ^ (sr & (NC - 1)))] = vv;
+  }
+  {
+    const float4* qsrc = reinterpret_cast<const float4*>(p.qhat + ((long long)b * p.Hq + g * G) * D);
+    float4* qdst = reinterpret_cast<float4*>(qs);
+    for (int e = tid; e < G * D / 4; e += kDecThreads) qdst[e] = __ldcg(qsrc + e);
   }
   __syncthreads();
-  // partial of this CTA (m = -inf, zeros when it held no key)
-  for (int e = tid; e < G * DP; e += 256) {
+  // logits: thread (key sr, heads hq0 + 8 m)
+  {
+    const int sr = tid & 63;
+    for (int h = tid >> 6; h < G; h += kDecThreads / 64) {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      const float* qr = qs + h * D;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        float kf[8];
+        load8(reinterpret_cast<const __nv_bfloat16*>(&ks[sr * NC + (c ^ (sr & (NC - 1)))]), kf);
+        a0 = fmaf(kf[0], qr[8 * c + 0], a0); a1 = fmaf(kf[1], qr[8 * c + 1], a1);
+        a2 = fmaf(kf[2], qr[8 * c + 2], a2); a3 = fmaf(kf[3], qr[8 * c + 3], a3);
+        a0 = fmaf(kf[4], qr[8 * c + 4], a0); a1 = fmaf(kf[5], qr[8 * c + 5], a1);
+        a2 = fmaf(kf[6], qr[8 * c + 6], a2); a3 = fmaf(kf[7], qr[8 * c + 7], a3);
+      }
+      lg[h * 64 + sr] = sr < nk ? ((a0 + a1) + (a2 + a3)) * p.sl2 : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // softmax of one block per head: one warp per head, two logits per lane
+  for (int h = warp; h < G; h += kDecWarps) {
+    const float x0 = lg[h * 64 + lane], x1 = lg[h * 64 + lane + 32];
+    const float m = warp_max(fmaxf(x0, x1));
+    const float p0 = exp2f(x0 - m), p1 = exp2f(x1 - m);
+    const float l = warp_sum(p0 + p1);
+    lg[h * 64 + lane] = p0;
+    lg[h * 64 + lane + 32] = p1;
+    if (lane == 0) { ml[2 * h] = m; ml[2 * h + 1] = l; }
+  }
+  __syncthreads();
+  // P V: item (head, 8-column chunk, key half)
+  for (int e = tid; e < G * NC * 2; e += kDecThreads) {
+    const int half = e & 1, c = (e >> 1) % NC, h = (e >> 1) / NC;
+    float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int s0 = half * 32, s1 = min(nk, s0 + 32);
+    for (int sr = s0; sr < s1; ++sr) {
+      float vf[8];
+      load8(reinterpret_cast<const __nv_bfloat16*>(&vs[sr * NC + (c ^ (sr & (NC - 1)))]), vf);
+      const float pr = lg[h * 64 + sr];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) o[w] = fmaf(pr, vf[w], o[w]);
+    }
+#pragma unroll
+    for (int w = 0; w < 8; ++w) red[(half * G + h) * D + 8 * c + w] = o[w];
+  }
+  __syncthreads();
+  for (int e = tid; e < G * DP; e += kDecThreads) {
     const int h = e / DP, c = e % DP;
-    pbase[e] = c == 0 ? ml[2 * h] : (c == 1 ? ml[2 * h + 1] : (c < 4 ? 0.f : os[h * D + c - 4]));
+    pb[e] = c == 0 ? ml[2 * h]
+                   : (c == 1 ? ml[2 * h + 1]
+                             : (c < 4 ? 0.f : red[h * D + c - 4] + red[(G + h) * D + c - 4]));
   }
 }
 
-// Combine of the n_parts partials of one q head and the output gate: one CTA
-// per (batch, q head), one thread per output column.
+// Combine of the `width` partials of q head hq of batch b and the output
+// gate.  Thread (quarter of the partials, column).
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
-decode_combine_kernel(const float* __restrict__ part, const T* __restrict__ gate,
-                      T* __restrict__ out, int Hq, int Hkv, int n_parts) {
+__device__ void dec_combine_unit(const DecodeParams& p, int u, float* sm) {
   constexpr int DP = D + 4;
-  extern __shared__ float wl[];                          // [n_parts] weights, [n_parts] sums
-  __shared__ float s_l;
-  const int hq = blockIdx.x % Hq;
-  const int b = blockIdx.x / Hq;
-  const int G = Hq / Hkv, g = hq / G, h = hq % G;
+  constexpr int NQ = kDecThreads / D;
+  const int hq = u % p.Hq, b = u / p.Hq;
+  const int G = p.Hq / p.Hkv, g = hq / G, h = hq % G;
   const int tid = threadIdx.x;
-  const float* pb = part + (((long long)b * Hkv + g) * n_parts * G + h) * DP;
+  float* wts = sm;                       // [width]
+  float* red = sm + p.width;             // [NQ][D]
+  __shared__ float s_l;
+  const float* pb = p.part + (((long long)b * p.Hkv + g) * p.width * G + h) * DP;
   const long long pstride = (long long)G * DP;
-  for (int e = tid; e < n_parts; e += D) {
-    wl[e] = pb[e * pstride];
-    wl[n_parts + e] = pb[e * pstride + 1];
-  }
-  __syncthreads();
   if (tid < 32) {
     float M = -INFINITY;
-    for (int e = tid; e < n_parts; e += 32) M = fmaxf(M, wl[e]);
+    for (int e = tid; e < p.width; e += 32) M = fmaxf(M, __ldcg(pb + e * pstride));
     M = warp_max(M);
     float L = 0.f;
-    for (int e = tid; e < n_parts; e += 32) {
-      const float f = wl[e] == -INFINITY ? 0.f : exp2f(wl[e] - M);
-      L = fmaf(f, wl[n_parts + e], L);
-      wl[e] = f;
+    for (int e = tid; e < p.width; e += 32) {
+      const float m = __ldcg(pb + e * pstride);
+      const float f = m == -INFINITY ? 0.f : exp2f(m - M);
+      L = fmaf(f, __ldcg(pb + e * pstride + 1), L);
+      wts[e] = f;
     }
     L = warp_sum(L);
     if (tid == 0) s_l = L;
   }
   __syncthreads();
-  // 8 independent partial sums so that the loads of 8 partials overlap
-  float o8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int e = 0;
-  for (; e + 8 <= n_parts; e += 8) {
+  const int col = tid % D, qtr = tid / D;
+  float o = 0.f;
+  for (int e = qtr; e < p.width; e += NQ) o = fmaf(wts[e], __ldcg(pb + e * pstride + 4 + col), o);
+  red[qtr * D + col] = o;
+  __syncthreads();
+  if (tid < D) {
+    float acc = 0.f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) o8[u] = fmaf(wl[e + u], pb[(e + u) * pstride + 4 + tid], o8[u]);
+    for (int r = 0; r < NQ; ++r) acc += red[r * D + tid];
+    const long long off = ((long long)b * p.Hq + hq) * D + tid;
+    const float inv = s_l > 0.f ? 1.f / s_l : 0.f;
+    static_cast<T*>(p.out)[off] = from_f32<T>(sigmoidf_(ldf<T>(p.gate, off)) * acc * inv);
   }
-  for (; e < n_parts; ++e) o8[0] = fmaf(wl[e], pb[e * pstride + 4 + tid], o8[0]);
-  const float o = ((o8[0] + o8[1]) + (o8[2] + o8[3])) + ((o8[4] + o8[5]) + (o8[6] + o8[7]));
-  const long long off = ((long long)b * Hq + hq) * D + tid;
-  out[off] = from_f32<T>(sigmoidf_(to_f32(gate[off])) * o / s_l);
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_step_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(16) unsigned char dec_smem[];
+  float* sm = reinterpret_cast<float*>(dec_smem);
+  __shared__ int scan_scratch[kDecThreads / 32 + 1];
+  const bool ranked = p.kk > 0 && p.kk < p.n_cand;
+  const int BG = p.B * p.Hkv;
+  const int n_score = ranked ? BG * p.n_chunks : 0;
+  const int n_lin = p.n_linear * p.B * p.H;
+
+  // P0: scores + histogram, linear layers, sparse prep
+  for (int u = blockIdx.x; u < n_score + n_lin + p.B; u += gridDim.x) {
+    if (u < n_score) dec_score_unit<T, D>(p, u, sm);
+    else if (u < n_score + n_lin) dec_linear_unit<T, D>(p, u - n_score, sm);
+    else dec_sparse_prep_unit<T, D>(p, u - n_score - n_lin);
+    __syncthreads();
+  }
+  if (!dec_grid_sync(p.ctl + 0, p.ctl + kDecCtlBarriers + 0, [&] {
+        if (ranked) dec_find_thresholds(p, scan_scratch);
+      }))
+    return;
+  // P1: emission and exact resolution (or direct rows)
+  const int n_p1 = ranked ? n_score : BG;
+  for (int u = blockIdx.x; u < n_p1; u += gridDim.x) {
+    if (ranked) dec_emit_unit<D>(p, u, dec_smem);
+    else dec_direct_row(p, u);
+    __syncthreads();
+  }
+  if (!dec_grid_sync(p.ctl + 1, p.ctl + kDecCtlBarriers + 1, [] {})) return;
+  // P2: attention partials
+  for (int u = blockIdx.x; u < BG * p.width; u += gridDim.x) {
+    dec_attn_unit<D>(p, u, dec_smem);
+    __syncthreads();
+  }
+  if (!dec_grid_sync(p.ctl + 2, p.ctl + kDecCtlBarriers + 2, [] {})) return;
+  // P3: combine and gate
+  for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {
+    dec_combine_unit<T, D>(p, u, sm);
+    __syncthreads();
+  }
+}
+
+// Dynamic shared memory of the step: the largest phase's need.
+inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int width) {
+  const size_t score = (size_t)(kDecWarps + 1) * D * 4;
+  const size_t lin = (size_t)(3 * D + kDecThreads) * 4;
+  const size_t attn = (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
+                      (size_t)2 * G * D * 4 + (size_t)G * 8;
+  const size_t resolve = (size_t)2 * topk * 4 + 16 +
+                         std::max((size_t)kDecBndMax * 8, (size_t)capb * 4);
+  const size_t comb = (size_t)width * 4 + (size_t)(kDecThreads / D) * D * 4;
+  return std::max(std::max(std::max(score, lin), std::max(attn, resolve)), comb);
 }
 
 }  // namespace sala

@@ -21,8 +21,11 @@ namespace sala {
 
 constexpr int kSelectThreads = 256;
 
+// Exclusive prefix sum of one int per thread over a CTA of NT threads
+// (NT / 32 <= 32); *total gets the sum.  scratch: >= NT/32 + 1 ints.
+template <int NT = kSelectThreads>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* total) {
-  // scratch: >= kSelectThreads/32 + 1 ints
+  static_assert(NT % 32 == 0 && NT / 32 <= 32, "one warp scans the warp totals");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -33,24 +36,25 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
   if (lane == 31) scratch[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < kSelectThreads / 32 ? scratch[lane] : 0;
+    int w = lane < NT / 32 ? scratch[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    if (lane < kSelectThreads / 32) scratch[lane] = w;   // inclusive per warp
+    if (lane < NT / 32) scratch[lane] = w;   // inclusive per warp
   }
   __syncthreads();
   const int before = (warp ? scratch[warp - 1] : 0) + x - v;
-  *total = scratch[kSelectThreads / 32 - 1];
+  *total = scratch[NT / 32 - 1];
   __syncthreads();
   return before;
 }
 
 // Top-k of n_cand keys held in shared memory (k < n_cand): writes the chosen
 // candidate numbers c (ascending) to out[0..k) as base + c.  Whole CTA of
-// kSelectThreads threads; hist / scan_scratch / s_prefix / s_need in smem.
+// NT threads; hist [256] / scan_scratch / s_prefix / s_need in smem.
+template <int NT = kSelectThreads>
 __device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_cand, int k,
                                                  int32_t* out, int base, int* hist,
                                                  int* scan_scratch, uint32_t* s_prefix,
@@ -60,9 +64,9 @@ __device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_can
   int need = k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int e = tid; e < 256; e += kSelectThreads) hist[e] = 0;
+    for (int e = tid; e < 256; e += NT) hist[e] = 0;
     __syncthreads();
-    for (int c = tid; c < n_cand; c += kSelectThreads) {
+    for (int c = tid; c < n_cand; c += NT) {
       const uint32_t key = keys[c];
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
@@ -101,7 +105,7 @@ __device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_can
   const uint32_t T = prefix;   // key of the k-th largest score; `need` ties at T are taken
 
   // ordered compaction: each thread owns a contiguous range of candidates
-  const int per = (n_cand + kSelectThreads - 1) / kSelectThreads;
+  const int per = (n_cand + NT - 1) / NT;
   const int lo = min(n_cand, tid * per), hi = min(n_cand, lo + per);
   int n_gt = 0, n_eq = 0;
   for (int c = lo; c < hi; ++c) {
@@ -110,9 +114,9 @@ __device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_can
     n_eq += key == T;
   }
   int tot;
-  const int eq_before = block_exclusive_scan(n_eq, scan_scratch, &tot);
+  const int eq_before = block_exclusive_scan<NT>(n_eq, scan_scratch, &tot);
   const int take_eq = max(0, min(n_eq, need - eq_before));
-  const int out_before = block_exclusive_scan(n_gt + take_eq, scan_scratch, &tot);
+  const int out_before = block_exclusive_scan<NT>(n_gt + take_eq, scan_scratch, &tot);
   int pos = out_before, eq_seen = 0;
   for (int c = lo; c < hi; ++c) {
     const uint32_t key = keys[c];

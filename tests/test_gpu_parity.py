@@ -313,3 +313,51 @@ def test_sparse_prefill_empty_index_row(sala, name, seqlen):
         sp.block, query_blocks=blocks)
     want[:, rows, :G] = 0.0
     assert rel_err(f64(out), want) <= TOL
+
+
+def test_decode_tied_scores_exact_fallback(sala):
+    """Every cached key is the same vector, so all 1098 candidate blocks score
+    exactly alike: the whole candidate set falls in one histogram bin, more
+    than the boundary list resolves by rank counting, and the step takes the
+    exact radix-select fallback.  Ties go to the lower block, as in the oracle."""
+    dev = torch.device("cuda")
+    w = _w("group_32k", sparse={"topk": 16, "n_local": 2})
+    sp, ln = w.sparse, w.linear
+    D, nblk = 128, 1100
+    N, cap = nblk * 64, nblk * 64 + 128
+    gen = torch.Generator(device=dev).manual_seed(11)
+    kvec = torch.randn((1, 1, sp.kv_heads, D), generator=gen, device=dev)
+    k = kvec.expand(1, N, sp.kv_heads, D).to(torch.bfloat16).contiguous()
+    v = torch.randn((1, N, sp.kv_heads, D), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.randn((1, N, sp.q_heads, D), generator=gen, device=dev).to(torch.bfloat16)
+    wt = wl.rms_weights(D, dev)
+    _, kn, kb, _ = sala.sparse_select(q, k, wt, wt, topk=sp.topk, n_init=sp.n_init,
+                                      n_local=sp.n_local)
+    k_cache = torch.zeros((1, cap, sp.kv_heads, D), dtype=torch.bfloat16, device=dev)
+    v_cache = torch.zeros_like(k_cache)
+    kbar = torch.zeros((1, cap // 64, sp.kv_heads, D), dtype=torch.float32, device=dev)
+    ksum = torch.zeros((1, sp.kv_heads, D), dtype=torch.float32, device=dev)
+    k_cache[:, :N] = kn
+    v_cache[:, :N] = v
+    kbar[:, :nblk] = kb
+    H = ln.heads
+    lam = lam_tensor(w, dev)
+    states = [torch.zeros((1, H, D, D), dtype=torch.float32, device=dev) for _ in range(w.n_linear)]
+    dd = sala.DecodeDesc(sala.linear_desc(1, 64, H, D),
+                         sala.sparse_desc(1, 64, sp.q_heads, sp.kv_heads, D, topk=sp.topk,
+                                          n_init=sp.n_init, n_local=sp.n_local),
+                         w.n_linear, cap)
+    ws = sala.workspace(sala.sala_decode_workspace_size(dd), dev)
+    tok = wl.decode_inputs(w, 0, dev)
+    outs = [torch.empty_like(t[0]) for t in tok]
+    io = sala.make_decode_io(tok, outs, states, [lam] * w.n_linear, wt, wt)
+    assert sala.sala_decode_step(dd, io, k_cache, v_cache, kbar, ksum, N, ws) == 0
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    tq, tk, tv, tg = (f64(t) for t in tok[w.n_linear])
+    k_hist = np.concatenate([f64(k), tk[:, None]], axis=1)
+    v_hist = np.concatenate([f64(v), tv[:, None]], axis=1)
+    ro, ridx = oracle.decode_sparse_step(k_hist, v_hist, tq, tg, f64(wt), f64(wt), N,
+                                         topk=sp.topk, n_init=sp.n_init, n_local=sp.n_local)
+    assert [int(j) for j in ridx[0, 0] if j >= 0][:sp.n_init + sp.topk] == list(range(17))
+    assert rel_err(f64(outs[w.n_linear]), ro) <= TOL
