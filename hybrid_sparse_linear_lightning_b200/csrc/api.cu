@@ -103,24 +103,29 @@ struct LinearWs {
 inline bool linear_on_tc(const sala_linear_desc* d) {
   return d->dtype == SALA_BF16 && d->head_dim == 128;
 }
+// Workspace: the tensor-core path (bf16, head_dim 128) normalises and rotates
+// Q and K inside its kernels and only needs the per-segment states; the
+// CUDA-core path keeps normalised bf16 copies of Q and K.
 LinearWs linear_ws(const sala_linear_desc* d) {
   const size_t n = (size_t)d->batch * d->seqlen * d->heads * d->head_dim;
   LinearWs w;
+  if (linear_on_tc(d)) {
+    const LinSegPlan p = lin_seg_plan(d->batch, d->heads, d->seqlen);
+    w.qn = w.kn = w.seg = 0;
+    w.total = align_up((size_t)d->batch * d->heads * p.n_seg * 128 * 128 * 4);
+    return w;
+  }
   w.qn = 0;
   w.kn = align_up(n * 2);
   w.seg = w.kn + align_up(n * 2);
   w.total = w.seg;
-  if (linear_on_tc(d)) {
-    const LinSegPlan p = lin_seg_plan(d->batch, d->heads, d->seqlen);
-    w.total += align_up((size_t)d->batch * d->heads * p.n_seg * 128 * 128 * 4);
-  }
   return w;
 }
 
-sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
-                           const __nv_bfloat16* kn, const void* v, const void* gate,
-                           const float* lambda, const float* state_in, float* state_out,
-                           void* out, float* seg_state, cudaStream_t st);
+sala_status run_linear_seg(const sala_linear_desc* d, const void* q, const void* k,
+                           const void* v, const void* gate, const float* lambda,
+                           const float* wq, const float* wk, const float* state_in,
+                           float* state_out, void* out, float* seg_state, cudaStream_t st);
 
 template <typename T, int D>
 sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, const void* v,
@@ -128,6 +133,12 @@ sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, 
                        const float* state_in, float* state_out, void* out, char* ws,
                        cudaStream_t st) {
   const LinearWs w = linear_ws(d);
+  // bf16 activations with head_dim 128 run on the tensor cores (norm and RoPE
+  // fused into the kernels); fp32 activations and head_dim 64 on CUDA cores
+  // after a separate norm / RoPE prologue.
+  if (std::is_same<T, __nv_bfloat16>::value && D == 128)
+    return run_linear_seg(d, q, k, v, gate, lambda, wq, wk, state_in, state_out, out,
+                          reinterpret_cast<float*>(ws + w.seg), st);
   auto* qn = reinterpret_cast<__nv_bfloat16*>(ws + w.qn);
   auto* kn = reinterpret_cast<__nv_bfloat16*>(ws + w.kn);
   const long long tokens = (long long)d->batch * d->seqlen;
@@ -136,11 +147,6 @@ sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, 
       static_cast<const T*>(q), static_cast<const T*>(k), wq, wk, qn, kn, tokens, d->seqlen,
       d->heads, d->pos0, rope_freq(D, d->rope_base), d->rms_eps);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
-  // bf16 activations with head_dim 128 run on the tensor cores; fp32
-  // activations and head_dim 64 on CUDA cores.
-  if (std::is_same<T, __nv_bfloat16>::value && D == 128)
-    return run_linear_seg(d, qn, kn, v, gate, lambda, state_in, state_out, out,
-                          reinterpret_cast<float*>(ws + w.seg), st);
   const size_t smem = sizeof(SimtSmem<D>);
   if (allow_smem(linear_chunk_simt_kernel<T, D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
   const int grid = d->batch * d->heads * (D / kSimtCols);
@@ -202,16 +208,17 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
-                           const __nv_bfloat16* kn, const void* v, const void* gate,
-                           const float* lambda, const float* state_in, float* state_out,
-                           void* out, float* seg_state, cudaStream_t st) {
+sala_status run_linear_seg(const sala_linear_desc* d, const void* q, const void* k,
+                           const void* v, const void* gate, const float* lambda,
+                           const float* wq, const float* wk, const float* state_in,
+                           float* state_out, void* out, float* seg_state, cudaStream_t st) {
   constexpr int D = 128;
   const LinSegPlan p = lin_seg_plan(d->batch, d->heads, d->seqlen);
   const uint64_t rows = (uint64_t)d->batch * d->seqlen, cols = (uint64_t)d->heads * D;
+  const RopeFreq rf = rope_freq(D, d->rope_base);
   CUtensorMap qm, km, vm, gm;
-  if (!make_tmap_bf16(&qm, qn, cols, rows, 64, kLsTile) ||
-      !make_tmap_bf16(&km, kn, cols, rows, 64, kLsTile) ||
+  if (!make_tmap_bf16(&qm, q, cols, rows, 64, kLsTile) ||
+      !make_tmap_bf16(&km, k, cols, rows, 64, kLsTile) ||
       !make_tmap_bf16(&vm, v, cols, rows, 64, kLsTile) ||
       !make_tmap_bf16(&gm, gate, cols, rows, 64, kLsTile))
     return SALA_ERR_CUDA;
@@ -219,8 +226,9 @@ sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
   // 1. segment sums
   const size_t smem_a = LsSumLayout::kBytes + 1024;
   if (allow_smem(linear_segsum_kernel, smem_a) != cudaSuccess) return SALA_ERR_CUDA;
-  linear_segsum_kernel<<<grid, kLsSumThreads, smem_a, st>>>(km, vm, lambda, seg_state, d->seqlen,
-                                                            d->heads, p.seg_tiles, p.n_seg);
+  linear_segsum_kernel<<<grid, kLsSumThreads, smem_a, st>>>(
+      km, vm, lambda, wk, d->rms_eps, d->pos0, rf, seg_state, d->seqlen, d->heads, p.seg_tiles,
+      p.n_seg);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
   // 2. scan over segments
   const long long n_el = (long long)d->batch * d->heads * D * D;
@@ -244,8 +252,9 @@ sala_status run_linear_seg(const sala_linear_desc* d, const __nv_bfloat16* qn,
   }
   if (regs_ok.load(std::memory_order_relaxed) != 1) return SALA_ERR_UNSUPPORTED;
   kern<<<grid, kLsOutThreads, smem_b, st>>>(qm, km, vm, gm, static_cast<const __nv_bfloat16*>(gate),
-                                            lambda, seg_state, static_cast<__nv_bfloat16*>(out),
-                                            d->seqlen, d->heads, p.seg_tiles, p.n_seg, d->scale);
+                                            lambda, wq, wk, d->rms_eps, d->pos0, rf, seg_state,
+                                            static_cast<__nv_bfloat16*>(out), d->seqlen, d->heads,
+                                            p.seg_tiles, p.n_seg, d->scale);
   return launch_status();
 }
 

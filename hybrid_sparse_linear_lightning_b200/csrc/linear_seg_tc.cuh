@@ -2,8 +2,12 @@
 // cores (bf16 activations, head_dim 128).
 //
 // Lightning attention (acgfav.com "SALA 混合架构": linear layers at O(N);
-// MiniCPM-SALA paper section 2.1: constant-size state).  With q^, k^
-// normalised and rotated, the state after token t is
+// MiniCPM-SALA paper section 2.1: constant-size state).  The kernels read the
+// RAW q and k tiles and apply QK-RMSNorm and RoPE in shared memory (QK
+// normalisation in every layer: MiniCPM-SALA paper, summary; RoPE kept in the
+// linear layers: acgfav.com "SALA 混合架构"), so the normalised tensors never
+// travel through HBM.  With q^, k^ normalised and rotated, the state after
+// token t is
 //   S_t = lam S_{t-1} + k^_t^T v_t,     o_t = scale * q^_t S_t,
 // so the state entering any token range is a decayed sum over everything
 // before it.  The sequence of every (batch, head) is cut into segments of
@@ -31,6 +35,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "prologue.cuh"
 #include "tc_ptx.cuh"
 
 namespace sala {
@@ -71,6 +76,55 @@ __device__ __forceinline__ void sw128_scale_row(uint8_t* tile, int r, float f) {
   }
 }
 
+// Row r of the same layout holds one token's raw q (or k) vector of one head
+// at position `pos`: replace it in place by
+//   f * RoPE(RMSNorm(x) * w, pos)
+// (RMSNorm over the 128 values, fp32; rotate-half RoPE, pairs (i, i + 64) =
+// chunk c of atom 0 and chunk c of atom 1 at the same swizzled offset).  The
+// angle pos * base^(-2i/128) is formed and reduced modulo 2 pi in fp64, then
+// evaluated by the special-function unit on [-pi, pi].
+__device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const float* __restrict__ w,
+                                                    float eps, long long pos, const RopeFreq& rf,
+                                                    float f) {
+  uint8_t* row0 = tile + r * 128;
+  uint8_t* row1 = tile + 16384 + r * 128;
+  float ss = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    const int o = (ch ^ (r & 7)) << 4;
+    float a[8], b[8];
+    load8(reinterpret_cast<const __nv_bfloat16*>(row0 + o), a);
+    load8(reinterpret_cast<const __nv_bfloat16*>(row1 + o), b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
+  }
+  const float rn = rsqrtf(ss * (1.0f / 128) + eps);
+  const double pd = (double)pos;
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+#pragma unroll 2
+  for (int ch = 0; ch < 8; ++ch) {
+    const int o = (ch ^ (r & 7)) << 4;
+    float a[8], b[8];
+    load8(reinterpret_cast<const __nv_bfloat16*>(row0 + o), a);
+    load8(reinterpret_cast<const __nv_bfloat16*>(row1 + o), b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = ch * 8 + e;
+      const float x1 = a[e] * rn * __ldg(w + i);
+      const float x2 = b[e] * rn * __ldg(w + 64 + i);
+      const double ang = pd * rf.inv[i];
+      const float red = (float)fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
+      float sn, cs;
+      __sincosf(red, &sn, &cs);
+      a[e] = (x1 * cs - x2 * sn) * f;
+      b[e] = (x2 * cs + x1 * sn) * f;
+    }
+    store8(reinterpret_cast<__nv_bfloat16*>(row0 + o), a);
+    store8(reinterpret_cast<__nv_bfloat16*>(row1 + o), b);
+  }
+}
+
 // 32 fp32 values -> bf16 columns [32 j, 32 j + 32) of row r of the same layout.
 __device__ __forceinline__ void sw128_store_row32(uint8_t* tile, int r, int j, const float* v) {
   uint8_t* atom = tile + (j >> 1) * 16384 + r * 128;
@@ -104,6 +158,8 @@ struct LsSumLayout {
 __global__ void __launch_bounds__(kLsSumThreads, 1)
 linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const float* __restrict__ lambda,
+                     const float* __restrict__ wk, float eps, long long pos0,
+                     const __grid_constant__ RopeFreq rf,
                      float* __restrict__ seg_state, int N, int H, int seg_tiles, int n_seg) {
   using L = LsSumLayout;
   constexpr int D = 128;
@@ -192,10 +248,11 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
       const int Lt = min(kLsTile, N - tile_start);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + st, (c / kLsSumStages) & 1));
       if (!ok) break;
-      // k_j scaled by lam^(seg_end - 1 - j) = lam^(seg_end - tile_end) lam^(L - 1 - r)
+      // k^_j (normalised, rotated at its position) scaled by
+      // lam^(seg_end - 1 - j) = lam^(seg_end - tile_end) lam^(L - 1 - r)
       const float ft = (float)pow((double)lam, (double)(seg_end - (tile_start + Lt)));
       const float f = r < Lt ? ft * pw[Lt - 1 - r] : 0.f;
-      sw128_scale_row(smem + st * L::kStage, r, f);
+      sw128_norm_rope_row(smem + st * L::kStage, r, wk, eps, pos0 + tile_start + r, rf, f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(k_ready + st);
@@ -278,8 +335,8 @@ struct LsOutLayout {
   static constexpr int kPw = kS + 32768;                 // lam^m, m = 0..128
   static constexpr int kBar = kPw + 4 * 132;
   // ld_full[2], ld_empty[2], qk_full, qk_empty, p_full, qk_scaled, s_scaled, s_full,
-  // s_smem_full, s_smem_empty, o_full[2], o_empty[2], fin
-  static constexpr int kNumBars = 4 + 8 + 4 + 1;
+  // s_smem_full, s_smem_empty, o_full[2], o_empty[2], fin, qk_ready
+  static constexpr int kNumBars = 4 + 8 + 4 + 1 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kBytes = kMisc + 16;
   // TMEM columns
@@ -291,10 +348,11 @@ struct LsOutLayout {
 // Warpgroup roles: warpgroup 0 holds the TMA producer (warp 0), the MMA
 // issuer (warp 1, one elected thread) and the TMEM owner (warp 2) and gives
 // registers away (56 per thread); warpgroups 1-3 take them (152 per thread):
-// warpgroup 1 rescales Q^ into Q' and builds P (one warp per TMEM lane
-// quadrant), warpgroup 2 rescales K^ into K' and carries the state (fp32 in
-// TMEM; a bf16 copy in shared memory is the B operand of the next Q' S
-// product),
+// warpgroup 1 normalises and rotates the raw Q rows of each tile in place,
+// then rescales Q^ into Q' and builds P (one warp per TMEM lane quadrant),
+// warpgroup 2 normalises and rotates the raw K rows, rescales K^ into K' and
+// carries the state (fp32 in TMEM; a bf16 copy in shared memory is the B
+// operand of the next Q' S product),
 // warpgroup 3 runs the gated epilogue of tile c while tile c + 1 accumulates
 // into the other O buffer.  56 x 128 + 152 x 384 = 65536 = 128 x 512, the
 // registers the block is launched with (the host checks the 128).
@@ -309,7 +367,9 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap,
                      const __grid_constant__ CUtensorMap gmap, const T* __restrict__ gate,
-                     const float* __restrict__ lambda, const float* __restrict__ seg_state,
+                     const float* __restrict__ lambda, const float* __restrict__ wq,
+                     const float* __restrict__ wk, float eps, long long pos0,
+                     const __grid_constant__ RopeFreq rf, const float* __restrict__ seg_state,
                      T* __restrict__ out, int N, int H, int seg_tiles, int n_seg, float scale) {
   using L = LsOutLayout;
   constexpr int D = 128;
@@ -330,6 +390,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* o_full = bars + 12;          // [2]
   uint64_t* o_empty = bars + 14;         // [2]
   uint64_t* fin = bars + 16;
+  uint64_t* qk_ready = bars + 17;        // raw Q and K of the tile normalised and rotated
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   float* pw = reinterpret_cast<float*>(smem + L::kPw);
 
@@ -360,6 +421,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::mbar_init(o_empty + i, 4);
     }
     tc::mbar_init(fin, 1);
+    tc::mbar_init(qk_ready, 8);
     tc::fence_barrier_init();
   }
   if (threadIdx.x <= kLsTile) pw[threadIdx.x] = (float)pow((double)lam, (double)threadIdx.x);
@@ -408,8 +470,9 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
           const int st = c & 1;
           const uint32_t q = base + st * L::kStage + L::kQ, k = base + st * L::kStage + L::kK,
                          v = base + st * L::kStage + L::kV;
-          // QK = Q^ K^T
+          // QK = Q^ K^T (raw tiles normalised and rotated in place first)
           if (!(ok = tc::mbar_wait(ld_full + st, (c >> 1) & 1))) break;
+          if (!(ok = tc::mbar_wait(qk_ready, c & 1))) break;
           if (c > 0 && !(ok = tc::mbar_wait(qk_empty, (c - 1) & 1))) break;
           tc::tc_fence_after();
   #pragma unroll
@@ -467,6 +530,13 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
     const int r = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     for (int c = 0; c < nt; ++c) {
+      // raw q row -> q^ (RMSNorm, RoPE at its position), in place
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1))) break;
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wq, eps,
+                          pos0 + (long long)(t0 + c) * kLsTile + r, rf, 1.f);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(qk_ready);
       if (!__all_sync(0xffffffffu, tc::mbar_wait(qk_full, c & 1))) break;
       // Q'_r = lam^(r+1) q^_r once Q^ K^T has read the tile
       sw128_scale_row(smem + (c & 1) * L::kStage + L::kQ, r, pw[r + 1]);
@@ -544,6 +614,14 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
     bool ok = true;
     for (int c = 0; ok && c < nt; ++c) {
       const int Lt = tile_len(c);
+      // raw k row -> k^ (RMSNorm, RoPE at its position), in place
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1));
+      if (!ok) break;
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wk, eps,
+                          pos0 + (long long)(t0 + c) * kLsTile + r, rf, 1.f);
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(qk_ready);
       // K'_r = lam^(L-1-r) k^_r (0 past the end) once Q^ K^T has read the tile
       ok = __all_sync(0xffffffffu, tc::mbar_wait(qk_full, c & 1));
       if (!ok) break;
