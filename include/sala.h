@@ -93,7 +93,11 @@ int sala_sparse_index_width(const sala_sparse_desc* d);
 
 size_t sala_linear_workspace_size(const sala_linear_desc* d);
 
-/* q, k, v, gate, out: [B, N, H, d] of d->dtype.  lambda: [H] fp32.
+/* One Lightning-style linear layer over N tokens (acgfav.com article, section
+ * "SALA 混合架构": linear layers at O(N); MiniCPM-SALA paper, section 2.1:
+ * constant-size state; QK normalisation and RoPE in these layers: paper
+ * summary and the HyPE sections of the articles).
+ * q, k, v, gate, out: [B, N, H, d] of d->dtype.  lambda: [H] fp32.
  * wq, wk: [d] fp32 RMSNorm weights.  state_in: [B, H, d, d] fp32 (row = key
  * dim, column = value dim) or NULL for zeros.  state_out: same layout, or
  * NULL; it may alias state_in.  workspace: >= sala_linear_workspace_size(d)
@@ -106,7 +110,9 @@ sala_status sala_linear_prefill(const sala_linear_desc* d, const void* q, const 
 
 size_t sala_sparse_workspace_size(const sala_sparse_desc* d);
 
-/* Selection stage of the sparse layer.
+/* Selection stage of the sparse layer (acgfav.com article, section
+ * "SALA 混合架构": a fine-grained block selection lets each query attend to a
+ * small set of key blocks; NoPE in the sparse layers under HyPE).
  * In:  q [B, N, Hq, d], k [B, N, Hkv, d] (d->dtype); wq, wk [d] fp32.
  * Out: q_norm [B, N, Hq, d] bf16 and k_norm [B, N, Hkv, d] bf16 (RMSNorm,
  *      no RoPE); kbar [B, N/block, Hkv, d] fp32 block means of the
@@ -145,12 +151,20 @@ sala_status sala_sparse_select_noalloc(const sala_sparse_desc* d, const void* q,
                                        const float* wq, const float* wk, void* q_norm,
                                        void* k_norm, float* kbar, int32_t* idx, void* stream);
 
-/* Gathered block-sparse attention with the sigmoid gate.
+/* Gathered block-sparse attention with the sigmoid gate (acgfav.com
+ * article, section "SALA 混合架构": exact attention of each query over its
+ * selected key blocks; MiniCPM-SALA paper, summary: an output gate after each
+ * attention block).
  * In:  q_norm [B, N, Hq, d] bf16, k_norm [B, N, Hkv, d] bf16 (as written by
  *      sala_sparse_select), v [B, N, Hkv, d] and gate [B, N, Hq, d] of
  *      d->dtype, idx as written by sala_sparse_select (entries >= 0 must be
- *      ascending block numbers <= the row's own block).
- * Out: out [B, N, Hq, d] of d->dtype. */
+ *      ascending block numbers <= the row's own block; a row must list at
+ *      least one block: an empty row gets a zero output and sets the bounds
+ *      bit of the status word).
+ * Out: out [B, N, Hq, d] of d->dtype.
+ * workspace / ws_bytes: reserved (ignored; may be NULL / 0).  The call needs
+ * no scratch today; the arguments keep the signature of the other prefill
+ * calls so that a future split of long index lists can use them. */
 sala_status sala_sparse_prefill(const sala_sparse_desc* d, const void* q_norm,
                                 const void* k_norm, const void* v, const void* gate,
                                 const int32_t* idx, void* out, void* workspace,
@@ -161,8 +175,11 @@ sala_status sala_sparse_prefill(const sala_sparse_desc* d, const void* q_norm,
 #define SALA_MAX_LAYERS 8
 
 /* One decode token through a layer group of n_linear linear layers followed
- * by one sparse layer.  lin.seqlen, lin.pos0 and sp.seqlen are ignored: the
- * new token sits at position cur_len. */
+ * by one sparse layer (MiniCPM-SALA paper, section 2.1: the linear layers
+ * carry a constant-size state; acgfav.com article, section "SALA 混合架构":
+ * the sparse layer's KV cache holds no position, so it is appended and
+ * scored as is).  lin.seqlen, lin.pos0 and sp.seqlen are ignored: the new
+ * token sits at position cur_len. */
 typedef struct {
   sala_linear_desc lin;
   sala_sparse_desc sp;
@@ -188,7 +205,10 @@ typedef struct {
 
 size_t sala_decode_workspace_size(const sala_decode_desc* d);
 
-/* k_cache, v_cache: [B, cache_capacity, Hkv, d] bf16; rows [0, cur_len) hold
+/* The step runs as ONE cooperative kernel launch (its CTAs synchronise
+ * through bounded grid barriers), preceded by a memset of the first bytes
+ * of the workspace; it can be captured in a CUDA graph.
+ * k_cache, v_cache: [B, cache_capacity, Hkv, d] bf16; rows [0, cur_len) hold
  * the normalised keys / raw values of the earlier tokens (the k_norm and v of
  * a prefill).  kbar: [B, cache_capacity/block, Hkv, d] fp32 block means of the
  * complete blocks (kbar of a prefill).  ksum: [B, Hkv, d] fp32 running sum of

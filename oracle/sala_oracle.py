@@ -64,6 +64,7 @@ __all__ = [
     "block_means", "block_scores", "select_row", "select_blocks",
     "selected_count", "sparse_attention", "sparse_select", "sparse_layer",
     "sparse_attention_rows", "sparse_select_rows", "sparse_layer_rows",
+    "token_softmax_importance", "select_token_softmax",
     "decode_linear_step", "decode_sparse_step",
 ]
 
@@ -360,6 +361,70 @@ def sparse_select_rows(q_rows, rows, k, wq, wk, *, block=64, topk=16, n_init=1, 
                 sel = select_row(scores[b, g, r], i, topk, n_init, n_local)
                 idx[b, g, r, : len(sel)] = sel
     return qh, kh, kbar, idx, scores
+
+
+def token_softmax_importance(qh_rows, kbar, rows, block, n_init, n_local):
+    """Block importance of the token-level selection variant.
+
+    Reading of the InfLLM-V2 block selection that the pages name (paper
+    summary and section 2.1; acgfav.com "SALA 混合架构": "fine-grained block
+    selection"): every query token t of query block i and every q head h of
+    kv group g scores each candidate key block j in [n_init, i - n_local]
+    against that block's mean normalised key, z = <q^_t^h, kbar_j^g> / sqrt(d);
+    the scores of one (token, head) are turned into a distribution over the
+    candidate blocks by a softmax; the importance of block j for query block
+    i is the probability mass all tokens of the block and all heads of the
+    group give it: I[b, g, r, j] = sum_{t in block rows[r]} sum_{h in G(g)}
+    softmax_j(z_t^h)(j).  Non-candidates are -inf.
+
+    qh_rows: [B, R*block, Hq, d] normalised queries of blocks rows[0..R);
+    kbar: [B, Hkv, nb, d].  Returns [B, Hkv, R, nb] (fp64).
+    """
+    qh_rows = np.asarray(qh_rows, F64)
+    kbar = np.asarray(kbar, F64)
+    B, _, Hq, d = qh_rows.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    G = Hq // Hkv
+    imp = np.full((B, Hkv, len(rows), nb), -np.inf, dtype=F64)
+    for b in range(B):
+        for g in range(Hkv):
+            for r, i in enumerate(rows):
+                cand = np.arange(n_init, i - n_local + 1)
+                if len(cand) == 0:
+                    continue
+                Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G].reshape(-1, d)
+                z = (Q @ kbar[b, g, cand].T) / math.sqrt(d)          # [T*G, C]
+                z = z - z.max(axis=1, keepdims=True)
+                p = np.exp(z)
+                p = p / p.sum(axis=1, keepdims=True)
+                imp[b, g, r, cand] = p.sum(axis=0)
+    return imp
+
+
+def select_token_softmax(q, k, wq, wk, *, block=64, topk=16, n_init=1, n_local=2, eps=1e-6,
+                         rows=None):
+    """Selection stage of the token-level variant (``token_softmax_importance``),
+    with the same initial / local blocks, top-k rule and tie-break as
+    ``select_row``.  Returns (q_hat, k_hat, kbar, idx, importance); ``rows``
+    restricts the work to those query blocks (importance rows then follow
+    ``rows``; idx keeps all nb rows, others -2)."""
+    qh = rms_norm(q, wq, eps)
+    kh = rms_norm(k, wk, eps)
+    kbar = block_means(kh, block)
+    B, N, Hq, d = qh.shape
+    nb = N // block
+    rs = list(range(nb)) if rows is None else [int(i) for i in rows]
+    q_rows = np.concatenate([qh[:, i * block:(i + 1) * block] for i in rs], axis=1)
+    imp = token_softmax_importance(q_rows, kbar, rs, block, n_init, n_local)
+    Hkv = kbar.shape[1]
+    idx = np.full((B, Hkv, nb, topk + n_init + n_local), -2, dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            for r, i in enumerate(rs):
+                sel = select_row(imp[b, g, r], i, topk, n_init, n_local)
+                idx[b, g, i, :] = -1
+                idx[b, g, i, : len(sel)] = sel
+    return qh, kh, kbar, idx, imp
 
 
 # ---------------------------------------------------------------------------

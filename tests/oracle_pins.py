@@ -291,6 +291,64 @@ def check_sparse_rows_forms(orc):
     assert _rel(kbar_r, kbar) < 1e-15 and _rel(qh_r, cat(qh)) < 1e-15
 
 
+def check_token_softmax_selection(orc):
+    # Token-level variant against an independent brute force: scalar loops
+    # for the scores, an explicit softmax per (token, head), the importance
+    # sums, and the best-scoring candidate subset by exhaustive search.
+    r = _rng(17)
+    B, blk, nb, Hq, Hkv, d = 1, 4, 9, 4, 2, 4
+    N = blk * nb
+    q = r.standard_normal((B, N, Hq, d))
+    k = r.standard_normal((B, N, Hkv, d))
+    w = np.ones(d)
+    topk, n_init, n_local = 2, 1, 2
+    _, _, _, idx, imp = orc.select_token_softmax(q, k, w, w, block=blk, topk=topk, n_init=n_init,
+                                                 n_local=n_local)
+    def nrm(x):
+        s_ = math.sqrt(sum(v * v for v in x) / len(x) + 1e-6)
+        return [v / s_ for v in x]
+    G = Hq // Hkv
+    for g in range(Hkv):
+        kb = []
+        for j in range(nb):
+            rows_ = [nrm(list(k[0, j * blk + t, g])) for t in range(blk)]
+            kb.append([sum(rr[e] for rr in rows_) / blk for e in range(d)])
+        for i in range(nb):
+            cand = list(range(n_init, i - n_local + 1))
+            tot = {j: 0.0 for j in cand}
+            for t in range(blk):
+                for h in range(g * G, (g + 1) * G):
+                    qq = nrm(list(q[0, i * blk + t, h]))
+                    z = {j: sum(qq[e] * kb[j][e] for e in range(d)) / math.sqrt(d) for j in cand}
+                    den = sum(math.exp(v) for v in z.values())
+                    for j in cand:
+                        tot[j] += math.exp(z[j]) / den
+            for j in cand:
+                assert abs(imp[0, g, i, j] - tot[j]) < 1e-12, (g, i, j)
+            best = ()
+            if cand:
+                best = max(itertools.combinations(cand, min(topk, len(cand))),
+                           key=lambda c: sum(tot[j] for j in c))
+            want = sorted(set(range(min(n_init, i + 1))) | set(range(max(0, i - n_local + 1), i + 1))
+                          | set(best))
+            assert [int(j) for j in idx[0, g, i] if j >= 0] == want, (g, i)
+
+
+def check_token_softmax_single_query(orc):
+    # One query token per block and one q head per kv head: the softmax is
+    # monotonic in the score, so the variant ranks candidates exactly as the
+    # block-mean rule does.
+    r = _rng(18)
+    q = r.standard_normal((1, 40, 2, 8))
+    k = r.standard_normal((1, 40, 2, 8))
+    w = np.ones(8)
+    kw = dict(block=1, topk=5, n_init=1, n_local=3)
+    _, _, _, idx_v, _ = orc.select_token_softmax(q, k, w, w, **kw)
+    _, _, _, idx_m, _ = orc.sparse_select(q, k, w, w, **kw)
+    assert np.array_equal(idx_v, idx_m)
+
+
+# --------------------------------------------------------------------------- sparse attention
 # --------------------------------------------------------------------------- sparse attention
 
 def _sdpa(q, k, v, mask=None, causal=False, scale=None):
@@ -398,6 +456,7 @@ ALL_CHECKS = [
     check_linear_special_lambdas, check_linear_segments, check_linear_layer_gate_rope,
     check_block_means_and_scores, check_selection_exhaustive, check_selection_ties,
     check_sparse_select_exhaustive, check_sparse_rows_forms,
+    check_token_softmax_selection, check_token_softmax_single_query,
     check_sparse_dense_limit, check_sparse_block_diagonal, check_sparse_masked_sdpa,
     check_decode_linear, check_decode_sparse,
 ]

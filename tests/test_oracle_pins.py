@@ -42,8 +42,10 @@ MUTANTS = [
     ("candidates overlap local", "lo, hi = n_init, b - n_local", "lo, hi = n_init, b - 1"),
     ("causal mask off by one", "mask = pos[None, :] <= t[:, None]", "mask = pos[None, :] < t[:, None] + 2"),
     ("softmax scale missing", "scale = 1.0 / math.sqrt(d)\n    o = np.empty(", "scale = 1.0\n    o = np.empty("),
-    ("sparse gqa mapping", "Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G]",
-     "Q = qh_rows[b, r * block:(r + 1) * block, g::Hkv]"),
+    ("sparse gqa mapping", "Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G]   # [T, G, d]",
+     "Q = qh_rows[b, r * block:(r + 1) * block, g::Hkv]   # [T, G, d]"),
+    ("token softmax gqa mapping", "Q = qh_rows[b, r * block:(r + 1) * block, g * G:(g + 1) * G].reshape(-1, d)",
+     "Q = qh_rows[b, r * block:(r + 1) * block, g::Hkv].reshape(-1, d)"),
     ("row scores ignore the block numbers", "qi = np.arange(nq) if rows is None else np.asarray(rows)",
      "qi = np.arange(nq)"),
     ("row attention uses the row number as the block", "t = np.arange(i * block, (i + 1) * block)",
@@ -54,6 +56,10 @@ MUTANTS = [
      "        np.einsum(\"bhk,bhv->bhkv\", kh, np.asarray(v, F64))",
      "S_new = lam[None, :, None, None] * (np.asarray(S, F64) + \\\n"
      "        np.einsum(\"bhk,bhv->bhkv\", kh, np.asarray(v, F64)))"),
+    ("token softmax over all blocks", "cand = np.arange(n_init, i - n_local + 1)\n                if len(cand) == 0:",
+     "cand = np.arange(0, i + 1)\n                if len(cand) == 0:"),
+    ("token importance without the softmax", "p = p / p.sum(axis=1, keepdims=True)\n                imp",
+     "p = z\n                imp"),
     ("decode query group sum", "qg = qh_s[b, gg * G:(gg + 1) * G].sum(axis=0, dtype=sd)",
      "qg = qh_s[b, gg * G]"),
 ]
