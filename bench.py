@@ -438,6 +438,63 @@ def per_config_entry(w, N, elapsed_ms, steps, per_call, peaks, ws, note=None):
 
 PER_CONFIG = [("group_32k", 10, False), ("group_128k", 5, False), ("group_1m", 3, True)]
 
+# fp32 FMA throughput of the CUDA cores: 148 SMs x 128 FMA lanes x 2 FLOP x
+# 1.965 GHz (unit counts and maximum clock of the B200)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def token_softmax_flops(w: wl.Workload, N: int) -> float:
+    """Work of the token-level selection variant: two passes (log-sum-exp,
+    then probabilities) of 2 * d FLOP per (query row, candidate block), over
+    64 * Hq query rows per query block, for the blocks that rank (fewer
+    slots than candidates)."""
+    sp = w.sparse
+    nb = N // sp.block
+    cand = 0
+    for i in range(nb):
+        n = max(0, i - sp.n_local + 1 - sp.n_init)
+        if 0 < min(sp.topk, n) < n:
+            cand += n
+    return 2.0 * 2 * sp.head_dim * sp.block * sp.q_heads * cand * w.batch
+
+
+def time_selection_variant(w: wl.Workload, dev, sala, steps: int = 5, warmup: int = 3):
+    """sala_sparse_select with SALA_SELECT_TOKEN_SOFTMAX on the workload's
+    sparse layer (CUDA events around each call)."""
+    sp = w.sparse
+    N = w.seqlen
+    q, k, _, _ = wl.layer_inputs(w, w.n_linear, dev)
+    wt = wl.rms_weights(sp.head_dim, dev)
+    d = sala.sparse_desc(w.batch, N, sp.q_heads, sp.kv_heads, sp.head_dim, sp.block, sp.topk,
+                         sp.n_init, sp.n_local, w.torch_dtype,
+                         selection=sala.SALA_SELECT_TOKEN_SOFTMAX)
+    nb = N // sp.block
+    outs = (torch.empty_like(q), torch.empty_like(k),
+            torch.empty((w.batch, nb, sp.kv_heads, sp.head_dim), dtype=torch.float32, device=dev),
+            torch.empty((w.batch, sp.kv_heads, nb, sala.sala_sparse_index_width(d)),
+                        dtype=torch.int32, device=dev))
+    wsp = sala.workspace(sala.sala_sparse_workspace_size(d), dev)
+    for _ in range(warmup):
+        assert sala.sala_sparse_select(d, q, k, wt, wt, *outs, wsp) == 0
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        assert sala.sala_sparse_select(d, q, k, wt, wt, *outs, wsp) == 0
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set in the selection variant")
+    ms = sum(a.elapsed_time(b) for a, b in ts) / steps
+    tf = token_softmax_flops(w, N) / (ms / 1e3) / 1e12
+    return {"workload": w.name, "selection": "token_softmax", "ms": round(ms, 4),
+            "bound": "alu", "achieved": round(tf, 2), "peak": round(FP32_ALU_TFLOPS, 1),
+            "unit": "TFLOP/s", "frac": round(tf / FP32_ALU_TFLOPS, 4),
+            "peak_source": "fp32 FMA lanes x SMs x max clock (no measured fp32 peak)"}
+
 
 def run_ours(args):
     rank, ws, local = dist_setup()
@@ -483,6 +540,11 @@ def run_ours(args):
                     "layer's normalised Q/K in the linear workspace (memory)") if lean else None
             per_config[name] = per_config_entry(wc, wc.seqlen, el, steps, pc, peaks, ws, note)
 
+    variants = None
+    if not args.no_per_config:
+        variants = [time_selection_variant(wl.WORKLOADS["group_32k"], dev, sala)]
+        torch.cuda.empty_cache()
+
     dec = None
     if args.decode_steps > 0:
         dec = run_decode(wl.WORKLOADS["group_1m"], args.decode_steps, dev, sala, peaks, ws)
@@ -510,7 +572,7 @@ def run_ours(args):
             "tensor_frac_of_step": round(sparse_attn_flops(w, N) / (ms_per_step / 1e3) / 1e12
                                          / peaks["bf16_tflops"], 4),
             "e2e": e2e, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
-            "per_config": per_config, "decode": dec,
+            "per_config": per_config, "selection_variants": variants, "decode": dec,
         }
         print(json.dumps(out), flush=True)
     if ws > 1:

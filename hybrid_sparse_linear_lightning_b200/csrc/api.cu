@@ -18,6 +18,7 @@
 #include "linear_seg_tc.cuh"
 #include "prologue.cuh"
 #include "select.cuh"
+#include "select_token.cuh"
 #include "sparse_simt.cuh"
 #include "sparse_tc.cuh"
 
@@ -68,6 +69,11 @@ sala_status check_sparse(const sala_sparse_desc* d) {
   if (d->block != 64 || d->seqlen % d->block != 0) return SALA_ERR_UNSUPPORTED;
   if (d->topk + d->n_init + d->n_local > 1024) return SALA_ERR_UNSUPPORTED;
   if (d->seqlen / d->block > 49152) return SALA_ERR_UNSUPPORTED;   // select smem: 4 B per block
+  if (d->selection != SALA_SELECT_BLOCK_MEAN && d->selection != SALA_SELECT_TOKEN_SOFTMAX)
+    return SALA_ERR_INVALID_ARG;
+  if (d->selection == SALA_SELECT_TOKEN_SOFTMAX &&
+      (d->seqlen / d->block > kTsMaxCand || d->q_heads / d->kv_heads > 64))
+    return SALA_ERR_UNSUPPORTED;
   return SALA_OK;
 }
 
@@ -167,9 +173,17 @@ sala_status run_select(const sala_sparse_desc* d, const void* q, const void* k, 
       static_cast<__nv_bfloat16*>(q_norm), static_cast<__nv_bfloat16*>(k_norm), qsum, kbar,
       d->seqlen, d->q_heads, d->kv_heads, d->block, d->rms_eps);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  const int width = d->topk + d->n_init + d->n_local;
+  if (d->selection == SALA_SELECT_TOKEN_SOFTMAX) {
+    const size_t ts_smem = TsLayout<D>::bytes(nb);
+    if (allow_smem(select_token_softmax_kernel<T, D>, ts_smem) != cudaSuccess) return SALA_ERR_CUDA;
+    select_token_softmax_kernel<T, D><<<d->batch * d->kv_heads * nb, kTsThreads, ts_smem, st>>>(
+        static_cast<const T*>(q), wq, kbar, idx, nb, d->q_heads, d->kv_heads, d->topk, d->n_init,
+        d->n_local, width, d->rms_eps);
+    return launch_status();
+  }
   const size_t smem = (size_t)nb * sizeof(uint32_t);
   if (allow_smem(select_topk_kernel<D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
-  const int width = d->topk + d->n_init + d->n_local;
   select_topk_kernel<D><<<d->batch * d->kv_heads * nb, kSelectThreads, smem, st>>>(
       qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width);
   return launch_status();
@@ -216,6 +230,8 @@ sala_status run_linear_seg(const sala_linear_desc* d, const void* q, const void*
   const LinSegPlan p = lin_seg_plan(d->batch, d->heads, d->seqlen);
   const uint64_t rows = (uint64_t)d->batch * d->seqlen, cols = (uint64_t)d->heads * D;
   const RopeFreq rf = rope_freq(D, d->rope_base);
+  RopeF32 rt;
+  for (int i = 0; i < 64; ++i) rt.th[i] = (float)rf.inv[i];
   CUtensorMap qm, km, vm, gm;
   if (!make_tmap_bf16(&qm, q, cols, rows, 64, kLsTile) ||
       !make_tmap_bf16(&km, k, cols, rows, 64, kLsTile) ||
@@ -227,7 +243,7 @@ sala_status run_linear_seg(const sala_linear_desc* d, const void* q, const void*
   const size_t smem_a = LsSumLayout::kBytes + 1024;
   if (allow_smem(linear_segsum_kernel, smem_a) != cudaSuccess) return SALA_ERR_CUDA;
   linear_segsum_kernel<<<grid, kLsSumThreads, smem_a, st>>>(
-      km, vm, lambda, wk, d->rms_eps, d->pos0, rf, seg_state, d->seqlen, d->heads, p.seg_tiles,
+      km, vm, lambda, wk, d->rms_eps, d->pos0, rf, rt, seg_state, d->seqlen, d->heads, p.seg_tiles,
       p.n_seg);
   if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
   // 2. scan over segments
@@ -252,7 +268,7 @@ sala_status run_linear_seg(const sala_linear_desc* d, const void* q, const void*
   }
   if (regs_ok.load(std::memory_order_relaxed) != 1) return SALA_ERR_UNSUPPORTED;
   kern<<<grid, kLsOutThreads, smem_b, st>>>(qm, km, vm, gm, static_cast<const __nv_bfloat16*>(gate),
-                                            lambda, wq, wk, d->rms_eps, d->pos0, rf, seg_state,
+                                            lambda, wq, wk, d->rms_eps, d->pos0, rf, rt, seg_state,
                                             static_cast<__nv_bfloat16*>(out), d->seqlen, d->heads,
                                             p.seg_tiles, p.n_seg, d->scale);
   return launch_status();
@@ -340,6 +356,7 @@ sala_status check_decode(const sala_decode_desc* d) {
   if (d->cache_capacity < d->sp.block || d->cache_capacity % d->sp.block != 0) return SALA_ERR_INVALID_ARG;
   if (d->cache_capacity / d->sp.block > 49152) return SALA_ERR_UNSUPPORTED;
   if (d->sp.q_heads > kDecodeMaxQHeads) return SALA_ERR_UNSUPPORTED;
+  if (d->sp.selection != SALA_SELECT_BLOCK_MEAN) return SALA_ERR_UNSUPPORTED;
   return SALA_OK;
 }
 

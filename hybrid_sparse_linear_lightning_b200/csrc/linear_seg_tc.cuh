@@ -76,15 +76,34 @@ __device__ __forceinline__ void sw128_scale_row(uint8_t* tile, int r, float f) {
   }
 }
 
-// Row r of the same layout holds one token's raw q (or k) vector of one head
-// at position `pos`: replace it in place by
-//   f * RoPE(RMSNorm(x) * w, pos)
+// RoPE frequencies base^(-2i/128), i < 64, rounded to fp32 (kernel parameter).
+struct RopeF32 {
+  float th[64];
+};
+
+// Base angles of a tile that starts at position p: lane l of the calling warp
+// returns (p * theta_l, p * theta_{l+32}) reduced modulo 2 pi, formed in fp64
+// (|p| < 2^53) and rounded to fp32.
+__device__ __forceinline__ float2 rope_tile_base(long long p, const RopeFreq& rf) {
+  const int lane = threadIdx.x & 31;
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+  const double a = (double)p * rf.inv[lane], b = (double)p * rf.inv[lane + 32];
+  return make_float2((float)fma(-rint(a * kInvTwoPi), kTwoPi, a),
+                     (float)fma(-rint(b * kInvTwoPi), kTwoPi, b));
+}
+
+// Row r of the same layout holds one token's raw q (or k) vector of one head,
+// at position (tile start + r): replace it in place by
+//   f * RoPE(RMSNorm(x) * w, position)
 // (RMSNorm over the 128 values, fp32; rotate-half RoPE, pairs (i, i + 64) =
 // chunk c of atom 0 and chunk c of atom 1 at the same swizzled offset).  The
-// angle pos * base^(-2i/128) is formed and reduced modulo 2 pi in fp64, then
-// evaluated by the special-function unit on [-pi, pi].
+// angle of frequency i is base_i + r * theta_i, with base_i (the tile start's
+// angle, reduced in fp64: rope_tile_base) taken from lane i % 32 of the
+// warp's `base`; it is reduced again to [-pi, pi] in fp32 (two-part 2 pi)
+// and evaluated by the special-function unit.  All 32 lanes must call this.
 __device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const float* __restrict__ w,
-                                                    float eps, long long pos, const RopeFreq& rf,
+                                                    float eps, float2 base, const RopeF32& rt,
                                                     float f) {
   uint8_t* row0 = tile + r * 128;
   uint8_t* row1 = tile + 16384 + r * 128;
@@ -99,10 +118,12 @@ __device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const 
     for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
   }
   const float rn = rsqrtf(ss * (1.0f / 128) + eps);
-  const double pd = (double)pos;
-  constexpr double kTwoPi = 6.283185307179586476925286766559;
-  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-#pragma unroll 2
+  const float rr = (float)r;
+  constexpr float kInvTwoPi = 0.159154943091895335768883763f;
+  constexpr float kTwoPiHi = 6.28318548202514648438f;        // 2 pi rounded to fp32
+  constexpr float kTwoPiLo = -1.74845553146951715461e-7f;    // 2 pi - kTwoPiHi
+  constexpr float kRound = 12582912.0f;                      // 1.5 * 2^23
+#pragma unroll
   for (int ch = 0; ch < 8; ++ch) {
     const int o = (ch ^ (r & 7)) << 4;
     float a[8], b[8];
@@ -113,8 +134,10 @@ __device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const 
       const int i = ch * 8 + e;
       const float x1 = a[e] * rn * __ldg(w + i);
       const float x2 = b[e] * rn * __ldg(w + 64 + i);
-      const double ang = pd * rf.inv[i];
-      const float red = (float)fma(-rint(ang * kInvTwoPi), kTwoPi, ang);
+      const float b0 = __shfl_sync(0xffffffffu, i < 32 ? base.x : base.y, i & 31);
+      const float ang = fmaf(rr, rt.th[i], b0);
+      const float n = fmaf(ang, kInvTwoPi, kRound) - kRound;   // nearest integer
+      const float red = fmaf(-n, kTwoPiLo, fmaf(-n, kTwoPiHi, ang));
       float sn, cs;
       __sincosf(red, &sn, &cs);
       a[e] = (x1 * cs - x2 * sn) * f;
@@ -159,7 +182,7 @@ __global__ void __launch_bounds__(kLsSumThreads, 1)
 linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const float* __restrict__ lambda,
                      const float* __restrict__ wk, float eps, long long pos0,
-                     const __grid_constant__ RopeFreq rf,
+                     const __grid_constant__ RopeFreq rf, const __grid_constant__ RopeF32 rt,
                      float* __restrict__ seg_state, int N, int H, int seg_tiles, int n_seg) {
   using L = LsSumLayout;
   constexpr int D = 128;
@@ -252,7 +275,8 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
       // lam^(seg_end - 1 - j) = lam^(seg_end - tile_end) lam^(L - 1 - r)
       const float ft = (float)pow((double)lam, (double)(seg_end - (tile_start + Lt)));
       const float f = r < Lt ? ft * pw[Lt - 1 - r] : 0.f;
-      sw128_norm_rope_row(smem + st * L::kStage, r, wk, eps, pos0 + tile_start + r, rf, f);
+      sw128_norm_rope_row(smem + st * L::kStage, r, wk, eps, rope_tile_base(pos0 + tile_start, rf),
+                          rt, f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(k_ready + st);
@@ -369,7 +393,8 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap gmap, const T* __restrict__ gate,
                      const float* __restrict__ lambda, const float* __restrict__ wq,
                      const float* __restrict__ wk, float eps, long long pos0,
-                     const __grid_constant__ RopeFreq rf, const float* __restrict__ seg_state,
+                     const __grid_constant__ RopeFreq rf, const __grid_constant__ RopeF32 rt,
+                     const float* __restrict__ seg_state,
                      T* __restrict__ out, int N, int H, int seg_tiles, int n_seg, float scale) {
   using L = LsOutLayout;
   constexpr int D = 128;
@@ -533,7 +558,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       // raw q row -> q^ (RMSNorm, RoPE at its position), in place
       if (!__all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1))) break;
       sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wq, eps,
-                          pos0 + (long long)(t0 + c) * kLsTile + r, rf, 1.f);
+                          rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, rf), rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qk_ready);
@@ -618,7 +643,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1));
       if (!ok) break;
       sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wk, eps,
-                          pos0 + (long long)(t0 + c) * kLsTile + r, rf, 1.f);
+                          rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, rf), rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qk_ready);

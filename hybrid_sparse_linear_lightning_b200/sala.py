@@ -26,6 +26,8 @@ SALA_ERR_WORKSPACE = 5
 SALA_ERR_DEVICE_FAULT = 6
 SALA_F32 = 0
 SALA_BF16 = 1
+SALA_SELECT_BLOCK_MEAN = 0
+SALA_SELECT_TOKEN_SOFTMAX = 1
 SALA_MAX_LAYERS = 8
 
 EXPORTED = [
@@ -55,7 +57,8 @@ class SparseDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("seqlen", ctypes.c_int), ("q_heads", ctypes.c_int),
                 ("kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("block", ctypes.c_int),
                 ("topk", ctypes.c_int), ("n_init", ctypes.c_int), ("n_local", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("rms_eps", ctypes.c_float), ("scale", ctypes.c_float)]
+                ("dtype", ctypes.c_int), ("rms_eps", ctypes.c_float), ("scale", ctypes.c_float),
+                ("selection", ctypes.c_int)]
 
 
 class DecodeDesc(ctypes.Structure):
@@ -143,9 +146,10 @@ def linear_desc(batch, seqlen, heads, head_dim, chunk=64, dtype=torch.bfloat16, 
 
 
 def sparse_desc(batch, seqlen, q_heads, kv_heads, head_dim, block=64, topk=16, n_init=1,
-                n_local=2, dtype=torch.bfloat16, rms_eps=1e-6, scale=0.0) -> SparseDesc:
+                n_local=2, dtype=torch.bfloat16, rms_eps=1e-6, scale=0.0,
+                selection=SALA_SELECT_BLOCK_MEAN) -> SparseDesc:
     return SparseDesc(batch, seqlen, q_heads, kv_heads, head_dim, block, topk, n_init, n_local,
-                      dtype_code(dtype), rms_eps, scale)
+                      dtype_code(dtype), rms_eps, scale, selection)
 
 
 # ---------------------------------------------------------------------------- raw entry points
@@ -249,11 +253,12 @@ def linear_prefill(q, k, v, gate, lam, wq, wk, *, chunk=64, pos0=0, rope_base=10
 
 
 def sparse_select(q, k, wq, wk, *, block=64, topk=16, n_init=1, n_local=2, rms_eps=1e-6,
-                  ws=None, outs=None, stream=None):
+                  selection=SALA_SELECT_BLOCK_MEAN, ws=None, outs=None, stream=None):
     """Selection stage; returns (q_norm, k_norm, kbar, idx)."""
     B, N, Hq, D = q.shape
     Hkv = k.shape[2]
-    d = sparse_desc(B, N, Hq, Hkv, D, block, topk, n_init, n_local, q.dtype, rms_eps)
+    d = sparse_desc(B, N, Hq, Hkv, D, block, topk, n_init, n_local, q.dtype, rms_eps,
+                    selection=selection)
     if outs is None:
         nb = N // block
         outs = (torch.empty((B, N, Hq, D), dtype=torch.bfloat16, device=q.device),

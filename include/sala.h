@@ -72,11 +72,21 @@ typedef struct {
   float scale;       /* 1.0                                                */
 } sala_linear_desc;
 
+/* How the sparse layer ranks its candidate blocks.
+ *   SALA_SELECT_BLOCK_MEAN: score_j = <sum_{h in group} qbar_b^h, kbar_j> / sqrt(d)
+ *     with qbar / kbar the block means of the normalised queries / keys.
+ *   SALA_SELECT_TOKEN_SOFTMAX: every query token t of block b and head h of
+ *     the group scores z = <q^_t^h, kbar_j> / sqrt(d); a softmax over the
+ *     candidate blocks makes it a distribution; importance_j = the summed
+ *     probability of all (t, h) (a reading of InfLLM-V2's block selection:
+ *     MiniCPM-SALA paper, summary and section 2.1).  Prefill selection only;
+ *     at most 8192 blocks (524288 tokens). */
+typedef enum { SALA_SELECT_BLOCK_MEAN = 0, SALA_SELECT_TOKEN_SOFTMAX = 1 } sala_selection;
+
 /* Sparse (InfLLM-V2-style) layer.  NoPE: RMSNorm only.  Blocks of `block`
  * tokens; query block b attends to the initial blocks [0, n_init), the local
  * blocks [b-n_local+1, b] and the top-`topk` candidate blocks in
- * [n_init, b-n_local], ranked by <sum_{h in group} qbar_b^h, kbar_j> / sqrt(d)
- * (block means of the normalised queries / keys; ties to the lower index).
+ * [n_init, b-n_local], ranked by `selection` (ties to the lower index).
  * Attention is exact softmax with logits * scale over the selected blocks'
  * keys at positions <= the query's.  scale <= 0 selects 1/sqrt(head_dim). */
 typedef struct {
@@ -84,6 +94,7 @@ typedef struct {
   sala_dtype dtype;
   float rms_eps;
   float scale;
+  sala_selection selection;   /* SALA_SELECT_BLOCK_MEAN (0) unless stated */
 } sala_sparse_desc;
 
 /* Width of one index row: topk + n_init + n_local. */

@@ -65,11 +65,11 @@ def test_linear_validation():
 
 def _sp(**kw):
     base = dict(batch=1, seqlen=2048, q_heads=4, kv_heads=1, head_dim=64, block=64, topk=4,
-                n_init=1, n_local=2)
+                n_init=1, n_local=2, selection=sala.SALA_SELECT_BLOCK_MEAN)
     base.update(kw)
     return sala.SparseDesc(base["batch"], base["seqlen"], base["q_heads"], base["kv_heads"],
                            base["head_dim"], base["block"], base["topk"], base["n_init"],
-                           base["n_local"], sala.SALA_BF16, 1e-6, 0.0)
+                           base["n_local"], sala.SALA_BF16, 1e-6, 0.0, base["selection"])
 
 
 def _call_select(d, ptr=FAKE, ws_bytes=1 << 40):
@@ -92,6 +92,10 @@ def test_sparse_validation():
     assert _call_select(d, ws_bytes=need - 1) == sala.SALA_ERR_WORKSPACE
     assert sala.LIB.sala_sparse_prefill(ctypes.byref(_sp(head_dim=80)), *([FAKE] * 6), None, 0,
                                         None) == sala.SALA_ERR_UNSUPPORTED
+    # selection rule: unknown value, token-softmax beyond its 8192-block limit
+    assert _call_select(_sp(selection=2)) == sala.SALA_ERR_INVALID_ARG
+    assert _call_select(_sp(selection=1, seqlen=64 * 8193)) == sala.SALA_ERR_UNSUPPORTED
+    assert sala.sala_sparse_workspace_size(_sp(selection=1)) > 0
 
 
 def test_decode_validation():
@@ -107,4 +111,6 @@ def test_decode_validation():
     bad = sala.DecodeDesc(_lin(), _sp(), 0, 4096)
     assert sala.sala_decode_workspace_size(bad) == 0
     bad = sala.DecodeDesc(_lin(), _sp(), 3, 100)      # capacity not a block multiple
+    assert sala.sala_decode_workspace_size(bad) == 0
+    bad = sala.DecodeDesc(_lin(), _sp(selection=1), 3, 4096)   # prefill-only selection rule
     assert sala.sala_decode_workspace_size(bad) == 0

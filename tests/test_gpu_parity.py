@@ -361,3 +361,31 @@ def test_decode_tied_scores_exact_fallback(sala):
                                          topk=sp.topk, n_init=sp.n_init, n_local=sp.n_local)
     assert [int(j) for j in ridx[0, 0] if j >= 0][:sp.n_init + sp.topk] == list(range(17))
     assert rel_err(f64(outs[w.n_linear]), ro) <= TOL
+
+
+@pytest.mark.parametrize("name,seqlen", [("tiny_2k_f32", 2048), ("group_32k", 4160)])
+def test_sparse_token_softmax_selection(sala, name, seqlen):
+    """Selection variant SALA_SELECT_TOKEN_SOFTMAX (per-token softmax over the
+    candidate blocks, probability mass summed over the block's tokens and the
+    group's heads) against the oracle's fp64 importance: index rows within
+    the tie window, then the whole layer's output over the GPU's lists."""
+    dev = torch.device("cuda")
+    w = wl.WORKLOADS[name]
+    sp = w.sparse
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev, seqlen=seqlen)
+    wt = wl.rms_weights(sp.head_dim, dev)
+    qn, kn, kbar, idx = sala.sparse_select(q, k, wt, wt, block=sp.block, topk=sp.topk,
+                                           n_init=sp.n_init, n_local=sp.n_local,
+                                           selection=sala.SALA_SELECT_TOKEN_SOFTMAX)
+    out = sala.sparse_prefill(qn, kn, v, g, idx, block=sp.block, topk=sp.topk, n_init=sp.n_init,
+                              n_local=sp.n_local)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    qh, kh, kb, ridx, imp = oracle.select_token_softmax(
+        f64(q), f64(k), f64(wt), f64(wt), block=sp.block, topk=sp.topk, n_init=sp.n_init,
+        n_local=sp.n_local)
+    gidx = idx.cpu().numpy()
+    n_tie = check_index_rows(gidx, ridx, imp, sp.topk, sp.n_init, sp.n_local)
+    assert n_tie <= max(1, gidx.shape[1] * gidx.shape[2] // 50), n_tie
+    want = oracle.sigmoid(f64(g)) * oracle.sparse_attention(qh, kh, f64(v), gidx, sp.block)
+    assert rel_err(f64(out), want) <= TOL
