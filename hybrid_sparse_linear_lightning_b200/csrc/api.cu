@@ -317,7 +317,7 @@ sala_status run_sparse_prefill(const sala_sparse_desc* d, const void* qn, const 
 }
 
 struct DecodeWs {
-  size_t ctl, hist, thr, keys, above, bnd, idx, qhat, part, total, zero_bytes;
+  size_t ctl, hist, keys, idx, qhat, part, total, zero_bytes;
 };
 DecodeWs decode_ws(const sala_decode_desc* d) {
   const sala_sparse_desc& s = d->sp;
@@ -328,12 +328,9 @@ DecodeWs decode_ws(const sala_decode_desc* d) {
   DecodeWs w;
   w.ctl = 0;
   w.hist = w.ctl + align_up(dec_ctl_words((int)BG) * 4);
-  w.thr = w.hist + align_up(BG * kDecBins * 4);
-  w.zero_bytes = w.thr;                          // control words and histograms
-  w.keys = w.thr + align_up(BG * 4);
-  w.above = w.keys + align_up(BG * capb * 4);
-  w.bnd = w.above + align_up(BG * std::max<size_t>(s.topk, 1) * 4);
-  w.idx = w.bnd + align_up(BG * kDecBndMax * 8);
+  w.keys = w.hist + align_up(BG * kDecBins * 4);
+  w.zero_bytes = w.keys;                         // control words and histograms
+  w.idx = w.keys + align_up(BG * capb * 4);
   w.qhat = w.idx + align_up(BG * width * 4);
   w.part = w.qhat + align_up(B * Hq * D * 4);
   w.total = w.part + align_up(BG * width * G * (D + 4) * 4);
@@ -408,10 +405,7 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   p.n_chunks = std::max(1, (p.n_cand + kDecChunk - 1) / kDecChunk);
   p.ctl = reinterpret_cast<unsigned*>(ws + w.ctl);
   p.hist = reinterpret_cast<unsigned*>(ws + w.hist);
-  p.thr = reinterpret_cast<unsigned*>(ws + w.thr);
   p.keys = reinterpret_cast<uint32_t*>(ws + w.keys);
-  p.above = reinterpret_cast<int*>(ws + w.above);
-  p.bnd = reinterpret_cast<uint2*>(ws + w.bnd);
   p.idx = reinterpret_cast<int*>(ws + w.idx);
   p.qhat = reinterpret_cast<float*>(ws + w.qhat);
   p.part = reinterpret_cast<float*>(ws + w.part);

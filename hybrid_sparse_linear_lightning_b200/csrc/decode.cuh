@@ -19,20 +19,20 @@
 //   P0  every linear (layer, batch, head) state update and output; the
 //       sparse layer's cache append and query normalisation; the scores of
 //       all candidate blocks in chunks of 256, each score also counted in a
-//       4096-bin histogram of its top 12 key bits per (batch, kv head).
-//   B1  the last CTA to arrive finds, per (batch, kv head), the bin T that
-//       holds the k-th largest score.
-//   P1  each chunk emits its candidates above bin T (certainly selected) and
-//       those in bin T (the boundary); the last chunk of a (batch, kv head)
-//       picks the remaining ones from the boundary exactly (score
-//       descending, ties to the lower block) and writes the ascending index
-//       list.  A boundary larger than 1024 entries (degenerate score
-//       distributions) falls back to an exact radix select over all scores.
-//   B2  barrier.
-//   P2  one unit per (batch, kv head, selected block): partial softmax sums
+//       4096-bin histogram of its top 12 key bits per (batch, kv head).  The
+//       CTA that scores the last chunk of a (batch, kv head) then selects
+//       for it while the other CTAs finish their units: the bin T holding
+//       the k-th largest score, the candidates above T (certainly selected)
+//       and those in T (the boundary), the remaining ones picked exactly from
+//       the boundary (score descending, ties to the lower block), and the
+//       ascending index row.  A boundary of more than 1024 entries
+//       (degenerate score distributions) falls back to an exact radix
+//       select over all scores.
+//   B1  barrier.
+//   P1  one unit per (batch, kv head, selected block): partial softmax sums
 //       of the group's q heads over that block's keys.
-//   B3  barrier.
-//   P3  one unit per (batch, q head): combine of the partials, output gate.
+//   B2  barrier.
+//   P2  one unit per (batch, q head): combine of the partials, output gate.
 //
 // Every wait is bounded (about a second); a barrier that runs out sets the
 // timeout bit of the status word and the CTAs return.
@@ -54,10 +54,18 @@ constexpr int kDecodeMaxQHeads = 64;    // largest sparse-layer q head count the
 constexpr int kDecMaxLayers = 8;
 
 // Control words at the start of the workspace (zeroed by the host before
-// each launch): barrier arrival counts, barrier release flags, and per
-// (batch, kv head) the above / boundary counts and the finished chunks.
-constexpr int kDecCtlBarriers = 4;
-__host__ __device__ constexpr int dec_ctl_words(int bg) { return 2 * kDecCtlBarriers + 4 * bg; }
+// each launch), each on its own 128-byte line: the barriers' arrival counts
+// and release flags, and per (batch, kv head) the number of scored chunks.
+constexpr int kDecCtlBarriers = 2;
+constexpr int kDecLine = 32;            // words per 128-byte line
+__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (2 * kDecCtlBarriers + bg); }
+__device__ __forceinline__ unsigned* dec_bar_count(unsigned* ctl, int i) { return ctl + kDecLine * i; }
+__device__ __forceinline__ unsigned* dec_bar_flag(unsigned* ctl, int i) {
+  return ctl + kDecLine * (kDecCtlBarriers + i);
+}
+__device__ __forceinline__ unsigned* dec_bg_done(unsigned* ctl, int bg) {
+  return ctl + kDecLine * (2 * kDecCtlBarriers + bg);
+}
 
 struct DecodeParams {
   // linear layers
@@ -92,10 +100,7 @@ struct DecodeParams {
   // workspace
   unsigned* ctl;
   unsigned* hist;       // [B * Hkv][kDecBins]
-  unsigned* thr;        // [B * Hkv]
   uint32_t* keys;       // [B * Hkv][capb]
-  int* above;           // [B * Hkv][topk]
-  uint2* bnd;           // [B * Hkv][kDecBndMax] (key, candidate)
   int* idx;             // [B * Hkv][width]
   float* qhat;          // [B][Hq][D]
   float* part;          // [B * Hkv][width][G][D + 4]
@@ -162,6 +167,9 @@ __device__ __forceinline__ float ldf(const void* p, long long i) {
 }
 
 // ------------------------------------------------------------------ P0 units
+
+template <int D>
+__device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem_raw);
 
 // Normalised query of q head h of batch b (RMSNorm over D, no rotation):
 // one warp, D/32 values per lane.
@@ -242,6 +250,18 @@ __device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
     const uint32_t key = score_key(s * rsqrtf((float)D));
     p.keys[(long long)bg * p.capb + c0 + c] = key;
     atomicAdd(p.hist + (long long)bg * kDecBins + (key >> (32 - kDecBinBits)), 1u);
+  }
+  // the CTA that finishes the last chunk of (b, g) selects for it
+  __shared__ int s_last_chunk;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last_chunk = atomicAdd(dec_bg_done(p.ctl, bg), 1u) == (unsigned)(p.n_chunks - 1);
+  }
+  __syncthreads();
+  if (s_last_chunk) {
+    __threadfence();
+    dec_select_bg<D>(p, bg, reinterpret_cast<unsigned char*>(sm));
   }
 }
 
@@ -358,57 +378,86 @@ __device__ void dec_sparse_prep_unit(const DecodeParams& p, int b) {
   }
 }
 
-// ------------------------------------------------------------------ B1, P1
+// ------------------------------------------------------------------ selection
 
-// Bin of the k-th largest key of every (batch, kv head): the last CTA at the
-// first barrier scans each 4096-bin histogram from the top.  Thread t owns
-// the 8 bins 4095 - 8t - u, u = 0..7.
-__device__ void dec_find_thresholds(const DecodeParams& p, int* scratch) {
-  static_assert(kDecBins == 8 * kDecThreads, "eight bins per thread");
+// Index row when no ranking is needed (no candidates, or k covers them all).
+__device__ void dec_direct_row(const DecodeParams& p, int bg) {
   const int tid = threadIdx.x;
-  for (int bg = 0; bg < p.B * p.Hkv; ++bg) {
+  const int b_ = p.bcur;
+  const int n_first = min(p.n_init, b_ + 1);
+  const int local_lo = max(p.n_init, b_ - p.n_local + 1);
+  const int n_loc = max(0, b_ - local_lo + 1);
+  int32_t* row = p.idx + (long long)bg * p.width;
+  for (int e = tid; e < n_first; e += kDecThreads) row[e] = e;
+  for (int e = tid; e < p.kk; e += kDecThreads) row[n_first + e] = p.n_init + e;
+  for (int e = tid; e < n_loc; e += kDecThreads) row[n_first + p.kk + e] = local_lo + e;
+  for (int e = n_first + p.kk + n_loc + tid; e < p.width; e += kDecThreads) row[e] = -1;
+}
+
+// Selection of (b, g) once all its scores and histogram counts are in, by
+// one CTA:
+//  1. T = the bin holding the kk-th largest key: the 4096 bins are scanned
+//     from the top (thread t owns bins 4095 - 8t - u, u = 0..7);
+//  2. every key above bin T is selected; the keys in bin T (the boundary)
+//     are collected with their candidate numbers;
+//  3. the remaining kk - n_above are the boundary entries of rank < that by
+//     (key descending, candidate ascending), found by counting;
+//  4. the kk candidates are ordered by counting and written, after the
+//     initial blocks and before the local ones.
+// If the boundary holds more than kDecBndMax entries, the kk candidates are
+// taken by an exact radix select over every key instead.
+template <int D>
+__device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem_raw) {
+  const int tid = threadIdx.x;
+  __shared__ int scan_s[kDecThreads / 32 + 1];
+  __shared__ int hist_s[256];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_need, s_T, s_n_above, s_n_bnd;
+  int32_t* chosen = reinterpret_cast<int32_t*>(smem_raw);          // [topk]
+  int32_t* sorted = chosen + p.topk;                               // [topk]
+  uint8_t* tail = reinterpret_cast<uint8_t*>(sorted + p.topk);
+  tail = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tail) + 15) & ~uintptr_t(15));
+  uint2* sb = reinterpret_cast<uint2*>(tail);                     // [kDecBndMax] boundary
+  // 1. threshold bin
+  {
     const unsigned* h = p.hist + (long long)bg * kDecBins;
     int cnt[8], tot = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) { cnt[u] = (int)__ldcg(h + kDecBins - 1 - 8 * tid - u); tot += cnt[u]; }
+    if (tid == 0) { s_n_above = 0; s_n_bnd = 0; s_T = 0; }
     int all;
-    const int before = block_exclusive_scan<kDecThreads>(tot, scratch, &all);
+    const int before = block_exclusive_scan<kDecThreads>(tot, scan_s, &all);
     if (before < p.kk && before + tot >= p.kk) {
       int cum = before, u = 0;
       for (; u < 8; ++u) {
         if (cum + cnt[u] >= p.kk) break;
         cum += cnt[u];
       }
-      p.thr[bg] = (unsigned)(kDecBins - 1 - 8 * tid - u);
+      s_T = kDecBins - 1 - 8 * tid - u;
     }
     __syncthreads();
   }
-}
-
-// Exact choice of the selected candidates of (b, g) once every chunk has
-// emitted: the `above` list plus the best (kk - n_above) boundary entries by
-// (key descending, candidate ascending), written as the ascending index row.
-template <int D>
-__device__ void dec_resolve(const DecodeParams& p, int bg, unsigned char* smem_raw) {
-  const int tid = threadIdx.x;
-  unsigned* ctl = p.ctl + 2 * kDecCtlBarriers + 4 * bg;
-  const int n_above = (int)min(ld_acquire_u32(ctl + 0), (unsigned)p.topk);
-  const int n_bnd = (int)ld_acquire_u32(ctl + 1);
+  // 2. above / boundary lists (slot order is arbitrary; the result is not)
+  const unsigned T = (unsigned)s_T;
+  for (int c = tid; c < p.n_cand; c += kDecThreads) {
+    const uint32_t key = __ldcg(p.keys + (long long)bg * p.capb + c);
+    const unsigned bin = key >> (32 - kDecBinBits);
+    if (bin > T) {
+      const int slot = atomicAdd(&s_n_above, 1);
+      if (slot < p.topk) chosen[slot] = c;
+      else set_status(kStatusBounds);
+    } else if (bin == T) {
+      const int slot = atomicAdd(&s_n_bnd, 1);
+      if (slot < kDecBndMax) sb[slot] = make_uint2(key, (unsigned)c);
+    }
+  }
+  __syncthreads();
+  const int n_above = min(s_n_above, p.topk);
+  const int n_bnd = s_n_bnd;
   const int need = p.kk - n_above;
-  int32_t* chosen = reinterpret_cast<int32_t*>(smem_raw);          // [topk]
-  int32_t* sorted = chosen + p.topk;                               // [topk]
-  uint8_t* tail = reinterpret_cast<uint8_t*>(sorted + p.topk);
-  tail = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tail) + 15) & ~uintptr_t(15));
-  __shared__ int hist_s[256];
-  __shared__ int scan_s[kDecThreads / 32 + 1];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_need;
   bool in_order = false;
   if (n_bnd <= kDecBndMax && need >= 1 && need <= n_bnd) {
-    uint2* sb = reinterpret_cast<uint2*>(tail);
-    for (int e = tid; e < n_above; e += kDecThreads) chosen[e] = __ldcg(p.above + (long long)bg * p.topk + e);
-    for (int e = tid; e < n_bnd; e += kDecThreads) sb[e] = __ldcg(p.bnd + (long long)bg * kDecBndMax + e);
-    __syncthreads();
+    // 3. ranks inside the boundary
     for (int e = tid; e < n_bnd; e += kDecThreads) {
       const uint2 me = sb[e];
       int rank = 0;
@@ -419,8 +468,9 @@ __device__ void dec_resolve(const DecodeParams& p, int bg, unsigned char* smem_r
       if (rank < need) chosen[n_above + rank] = (int)me.y;
     }
   } else {
-    // degenerate boundary: exact radix select over every score of (b, g)
+    // degenerate boundary: exact radix select over every key of (b, g)
     uint32_t* sk = reinterpret_cast<uint32_t*>(tail);
+    __syncthreads();
     for (int e = tid; e < p.n_cand; e += kDecThreads) sk[e] = __ldcg(p.keys + (long long)bg * p.capb + e);
     __syncthreads();
     topk_emit_sorted<kDecThreads>(sk, p.n_cand, p.kk, sorted, 0, hist_s, scan_s, &s_prefix,
@@ -437,6 +487,7 @@ __device__ void dec_resolve(const DecodeParams& p, int bg, unsigned char* smem_r
     }
     __syncthreads();
   }
+  // 4. the row
   const int b_ = p.bcur;
   const int n_first = min(p.n_init, b_ + 1);
   const int local_lo = max(p.n_init, b_ - p.n_local + 1);
@@ -448,55 +499,7 @@ __device__ void dec_resolve(const DecodeParams& p, int bg, unsigned char* smem_r
   for (int e = n_first + p.kk + n_loc + tid; e < p.width; e += kDecThreads) row[e] = -1;
 }
 
-// Index row when no ranking is needed (no candidates, or k covers them all).
-__device__ void dec_direct_row(const DecodeParams& p, int bg) {
-  const int tid = threadIdx.x;
-  const int b_ = p.bcur;
-  const int n_first = min(p.n_init, b_ + 1);
-  const int local_lo = max(p.n_init, b_ - p.n_local + 1);
-  const int n_loc = max(0, b_ - local_lo + 1);
-  int32_t* row = p.idx + (long long)bg * p.width;
-  for (int e = tid; e < n_first; e += kDecThreads) row[e] = e;
-  for (int e = tid; e < p.kk; e += kDecThreads) row[n_first + e] = p.n_init + e;
-  for (int e = tid; e < n_loc; e += kDecThreads) row[n_first + p.kk + e] = local_lo + e;
-  for (int e = n_first + p.kk + n_loc + tid; e < p.width; e += kDecThreads) row[e] = -1;
-}
-
-template <int D>
-__device__ void dec_emit_unit(const DecodeParams& p, int u, unsigned char* smem_raw) {
-  const int ck = u % p.n_chunks;
-  const int bg = u / p.n_chunks;
-  const int tid = threadIdx.x;
-  unsigned* ctl = p.ctl + 2 * kDecCtlBarriers + 4 * bg;
-  const unsigned T = __ldcg(p.thr + bg);
-  const int c0 = ck * kDecChunk;
-  const int nc = min(kDecChunk, p.n_cand - c0);
-  for (int c = tid; c < nc; c += kDecThreads) {
-    const uint32_t key = __ldcg(p.keys + (long long)bg * p.capb + c0 + c);
-    const unsigned bin = key >> (32 - kDecBinBits);
-    if (bin > T) {
-      const unsigned slot = atomicAdd(ctl + 0, 1u);
-      if (slot < (unsigned)p.topk) p.above[(long long)bg * p.topk + slot] = c0 + c;
-      else set_status(kStatusBounds);
-    } else if (bin == T) {
-      const unsigned slot = atomicAdd(ctl + 1, 1u);
-      if (slot < (unsigned)kDecBndMax) p.bnd[(long long)bg * kDecBndMax + slot] = make_uint2(key, c0 + c);
-    }
-  }
-  __shared__ int s_last_chunk;
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    s_last_chunk = atomicAdd(ctl + 2, 1u) == (unsigned)(p.n_chunks - 1);
-  }
-  __syncthreads();
-  if (s_last_chunk) {
-    __threadfence();
-    dec_resolve<D>(p, bg, smem_raw);
-  }
-}
-
-// ------------------------------------------------------------------ P2, P3
+// ------------------------------------------------------------------ P1, P2
 
 // Partial softmax sums of the G q heads of (b, g) over selected block `slot`:
 // [G][D + 4] = (m, l, -, -, o[D]) with logits in base 2.  Keys and values are
@@ -650,38 +653,29 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 decode_step_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(16) unsigned char dec_smem[];
   float* sm = reinterpret_cast<float*>(dec_smem);
-  __shared__ int scan_scratch[kDecThreads / 32 + 1];
   const bool ranked = p.kk > 0 && p.kk < p.n_cand;
   const int BG = p.B * p.Hkv;
   const int n_score = ranked ? BG * p.n_chunks : 0;
   const int n_lin = p.n_linear * p.B * p.H;
 
-  // P0: scores + histogram, linear layers, sparse prep
-  for (int u = blockIdx.x; u < n_score + n_lin + p.B; u += gridDim.x) {
+  // P0: scores + histogram (+ selection by the last chunk of each (b, g)),
+  // linear layers, sparse prep; direct index rows when nothing ranks
+  const int n_direct = ranked ? 0 : BG;
+  for (int u = blockIdx.x; u < n_score + n_lin + p.B + n_direct; u += gridDim.x) {
     if (u < n_score) dec_score_unit<T, D>(p, u, sm);
     else if (u < n_score + n_lin) dec_linear_unit<T, D>(p, u - n_score, sm);
-    else dec_sparse_prep_unit<T, D>(p, u - n_score - n_lin);
+    else if (u < n_score + n_lin + p.B) dec_sparse_prep_unit<T, D>(p, u - n_score - n_lin);
+    else dec_direct_row(p, u - n_score - n_lin - p.B);
     __syncthreads();
   }
-  if (!dec_grid_sync(p.ctl + 0, p.ctl + kDecCtlBarriers + 0, [&] {
-        if (ranked) dec_find_thresholds(p, scan_scratch);
-      }))
-    return;
-  // P1: emission and exact resolution (or direct rows)
-  const int n_p1 = ranked ? n_score : BG;
-  for (int u = blockIdx.x; u < n_p1; u += gridDim.x) {
-    if (ranked) dec_emit_unit<D>(p, u, dec_smem);
-    else dec_direct_row(p, u);
-    __syncthreads();
-  }
-  if (!dec_grid_sync(p.ctl + 1, p.ctl + kDecCtlBarriers + 1, [] {})) return;
-  // P2: attention partials
+  if (!dec_grid_sync(dec_bar_count(p.ctl, 0), dec_bar_flag(p.ctl, 0), [] {})) return;
+  // P1: attention partials
   for (int u = blockIdx.x; u < BG * p.width; u += gridDim.x) {
     dec_attn_unit<D>(p, u, dec_smem);
     __syncthreads();
   }
-  if (!dec_grid_sync(p.ctl + 2, p.ctl + kDecCtlBarriers + 2, [] {})) return;
-  // P3: combine and gate
+  if (!dec_grid_sync(dec_bar_count(p.ctl, 1), dec_bar_flag(p.ctl, 1), [] {})) return;
+  // P2: combine and gate
   for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {
     dec_combine_unit<T, D>(p, u, sm);
     __syncthreads();
@@ -695,7 +689,7 @@ inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int widt
   const size_t attn = (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
                       (size_t)2 * G * D * 4 + (size_t)G * 8;
   const size_t resolve = (size_t)2 * topk * 4 + 16 +
-                         std::max((size_t)kDecBndMax * 8, (size_t)capb * 4);
+                         std::max((size_t)kDecBndMax * 8, (size_t)capb * 4);   // dec_select_bg
   const size_t comb = (size_t)width * 4 + (size_t)(kDecThreads / D) * D * 4;
   return std::max(std::max(std::max(score, lin), std::max(attn, resolve)), comb);
 }

@@ -96,13 +96,15 @@ __device__ __forceinline__ float2 rope_tile_base(long long p, const RopeFreq& rf
 // Row r of the same layout holds one token's raw q (or k) vector of one head,
 // at position (tile start + r): replace it in place by
 //   f * RoPE(RMSNorm(x) * w, position)
-// (RMSNorm over the 128 values, fp32; rotate-half RoPE, pairs (i, i + 64) =
-// chunk c of atom 0 and chunk c of atom 1 at the same swizzled offset).  The
-// angle of frequency i is base_i + r * theta_i, with base_i (the tile start's
-// angle, reduced in fp64: rope_tile_base) taken from lane i % 32 of the
-// warp's `base`; it is reduced again to [-pi, pi] in fp32 (two-part 2 pi)
-// and evaluated by the special-function unit.  All 32 lanes must call this.
-__device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const float* __restrict__ w,
+// (RMSNorm over the 128 values, fp32, with the weights w [128] in shared
+// memory; rotate-half RoPE, pairs (i, i + 64) = chunk c of atom 0 and chunk
+// c of atom 1 at the same swizzled offset).  The angle of frequency i is
+// base_i + r * theta_i, with base_i (the tile start's angle, reduced in fp64:
+// rope_tile_base) taken from lane i % 32 of the warp's `base`; it lies in
+// [-pi, pi + 127], where the special-function unit's sine and cosine are
+// accurate to about 1e-6 without a further reduction.  All 32 lanes must
+// call this.
+__device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const float* wsm,
                                                     float eps, float2 base, const RopeF32& rt,
                                                     float f) {
   uint8_t* row0 = tile + r * 128;
@@ -117,31 +119,27 @@ __device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const 
 #pragma unroll
     for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
   }
-  const float rn = rsqrtf(ss * (1.0f / 128) + eps);
+  const float sc = rsqrtf(ss * (1.0f / 128) + eps) * f;
   const float rr = (float)r;
-  constexpr float kInvTwoPi = 0.159154943091895335768883763f;
-  constexpr float kTwoPiHi = 6.28318548202514648438f;        // 2 pi rounded to fp32
-  constexpr float kTwoPiLo = -1.74845553146951715461e-7f;    // 2 pi - kTwoPiHi
-  constexpr float kRound = 12582912.0f;                      // 1.5 * 2^23
 #pragma unroll
   for (int ch = 0; ch < 8; ++ch) {
     const int o = (ch ^ (r & 7)) << 4;
-    float a[8], b[8];
+    float a[8], b[8], wa[8], wb[8];
     load8(reinterpret_cast<const __nv_bfloat16*>(row0 + o), a);
     load8(reinterpret_cast<const __nv_bfloat16*>(row1 + o), b);
+    load8(wsm + ch * 8, wa);
+    load8(wsm + 64 + ch * 8, wb);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = ch * 8 + e;
-      const float x1 = a[e] * rn * __ldg(w + i);
-      const float x2 = b[e] * rn * __ldg(w + 64 + i);
+      const float x1 = a[e] * wa[e], x2 = b[e] * wb[e];
       const float b0 = __shfl_sync(0xffffffffu, i < 32 ? base.x : base.y, i & 31);
-      const float ang = fmaf(rr, rt.th[i], b0);
-      const float n = fmaf(ang, kInvTwoPi, kRound) - kRound;   // nearest integer
-      const float red = fmaf(-n, kTwoPiLo, fmaf(-n, kTwoPiHi, ang));
       float sn, cs;
-      __sincosf(red, &sn, &cs);
-      a[e] = (x1 * cs - x2 * sn) * f;
-      b[e] = (x2 * cs + x1 * sn) * f;
+      __sincosf(fmaf(rr, rt.th[i], b0), &sn, &cs);
+      cs *= sc;
+      sn *= sc;
+      a[e] = fmaf(x1, cs, -x2 * sn);
+      b[e] = fmaf(x2, cs, x1 * sn);
     }
     store8(reinterpret_cast<__nv_bfloat16*>(row0 + o), a);
     store8(reinterpret_cast<__nv_bfloat16*>(row1 + o), b);
@@ -166,7 +164,7 @@ __device__ __forceinline__ void sw128_store_row32(uint8_t* tile, int r, int j, c
 // 1. Segment sums
 // --------------------------------------------------------------------------
 
-constexpr int kLsSumThreads = 256;
+constexpr int kLsSumThreads = 512;     // warps 0-3: TMA, MMA, TMEM; 4-15: one scaling WG per stage
 constexpr int kLsSumStages = 3;
 
 struct LsSumLayout {
@@ -175,7 +173,8 @@ struct LsSumLayout {
   static constexpr int kPw = kLsSumStages * kStage;  // lam^m, m = 0..128
   static constexpr int kBar = kPw + 4 * 132;         // ld_full[S], ld_empty[S], k_ready[S], done
   static constexpr int kMisc = kBar + 8 * (3 * kLsSumStages + 1);
-  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kW = kMisc + 16;              // RMSNorm weights of k, 128 floats
+  static constexpr int kBytes = kW + 512;
 };
 
 __global__ void __launch_bounds__(kLsSumThreads, 1)
@@ -196,6 +195,7 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
   uint64_t* done = bars + 3 * kLsSumStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   float* pw = reinterpret_cast<float*>(smem + L::kPw);
+  float* wsm = reinterpret_cast<float*>(smem + L::kW);
 
   const int s = blockIdx.x % n_seg;
   const int h = (blockIdx.x / n_seg) % H;
@@ -217,6 +217,7 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
     tc::fence_barrier_init();
   }
   if (threadIdx.x <= kLsTile) pw[threadIdx.x] = (float)pow((double)lam, (double)threadIdx.x);
+  if (threadIdx.x < D) wsm[threadIdx.x] = wk[threadIdx.x];
   if (warp == 2) {
     tc::tmem_alloc(tmem_slot, 128);
     tc::tmem_relinquish();
@@ -262,11 +263,13 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
       tc::mma_commit(done);
     }
   } else if (warp >= 4) {
+    // scaling warpgroup a handles the tiles of stage a (c = a, a + 3, ...)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
+    const int a = (warp - 4) >> 2;
     bool ok = true;
-    for (int c = 0; ok && c < nt; ++c) {
-      const int st = c % kLsSumStages;
+    for (int c = a; ok && c < nt; c += kLsSumStages) {
+      const int st = a;
       const int tile_start = (t0 + c) * kLsTile;
       const int Lt = min(kLsTile, N - tile_start);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + st, (c / kLsSumStages) & 1));
@@ -275,14 +278,14 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
       // lam^(seg_end - 1 - j) = lam^(seg_end - tile_end) lam^(L - 1 - r)
       const float ft = (float)pow((double)lam, (double)(seg_end - (tile_start + Lt)));
       const float f = r < Lt ? ft * pw[Lt - 1 - r] : 0.f;
-      sw128_norm_rope_row(smem + st * L::kStage, r, wk, eps, rope_tile_base(pos0 + tile_start, rf),
+      sw128_norm_rope_row(smem + st * L::kStage, r, wsm, eps, rope_tile_base(pos0 + tile_start, rf),
                           rt, f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(k_ready + st);
     }
-    // dS (row r = key dim, 128 value columns) -> seg_state
-    if (__all_sync(0xffffffffu, ok && tc::mbar_wait(done, 0))) {
+    // dS (row r = key dim, 128 value columns) -> seg_state, by warpgroup 0
+    if (a == 0 && __all_sync(0xffffffffu, ok && tc::mbar_wait(done, 0))) {
       tc::tc_fence_after();
       float* dst = seg_state + ((((long long)b * H + h) * n_seg + s) * D + r) * D;
       const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -362,7 +365,8 @@ struct LsOutLayout {
   // s_smem_full, s_smem_empty, o_full[2], o_empty[2], fin, qk_ready
   static constexpr int kNumBars = 4 + 8 + 4 + 1 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
-  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kW = kMisc + 16;                  // RMSNorm weights of q, k: 2 x 128 floats
+  static constexpr int kBytes = kW + 1024;
   // TMEM columns
   static constexpr int kColQK = 0;     // Q^ K^T; P (bf16 pairs) overwrites its first 64 columns
   static constexpr int kColO = 128;    // O of tile c in columns 128 + 128 (c & 1)
@@ -418,6 +422,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* qk_ready = bars + 17;        // raw Q and K of the tile normalised and rotated
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   float* pw = reinterpret_cast<float*>(smem + L::kPw);
+  float* wsm = reinterpret_cast<float*>(smem + L::kW);   // [0, 128): wq, [128, 256): wk
 
   const int s = blockIdx.x % n_seg;
   const int h = (blockIdx.x / n_seg) % H;
@@ -450,6 +455,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
     tc::fence_barrier_init();
   }
   if (threadIdx.x <= kLsTile) pw[threadIdx.x] = (float)pow((double)lam, (double)threadIdx.x);
+  if (threadIdx.x < 2 * D) wsm[threadIdx.x] = threadIdx.x < D ? wq[threadIdx.x] : wk[threadIdx.x - D];
   if (warp == 2) {
     tc::tmem_alloc(tmem_slot, 512);
     tc::tmem_relinquish();
@@ -557,7 +563,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
     for (int c = 0; c < nt; ++c) {
       // raw q row -> q^ (RMSNorm, RoPE at its position), in place
       if (!__all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1))) break;
-      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wq, eps,
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wsm, eps,
                           rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, rf), rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
@@ -642,7 +648,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       // raw k row -> k^ (RMSNorm, RoPE at its position), in place
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1));
       if (!ok) break;
-      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wk, eps,
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wsm + D, eps,
                           rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, rf), rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
