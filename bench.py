@@ -30,6 +30,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
 
 from hybrid_sparse_linear_lightning_b200 import workloads as wl  # noqa: E402
 
@@ -212,6 +213,89 @@ class GroupPrefill:
             if timed_calls is not None:
                 e1.record()
                 timed_calls.append((name, e0, e1))
+
+
+class ShardedGroupPrefill:
+    """One rank's head shard of a layer group (``--shard heads``): linear
+    heads [lo, hi) of every linear layer and the q heads of its sparse-layer
+    shard, with the kv group's block-mean query sums all-reduced over NCCL
+    where a group spans several ranks.  Inputs are the rank's slices of the
+    seeded full tensors (each drawn in full, sliced, then freed)."""
+
+    def __init__(self, w: wl.Workload, N: int, dev, rank: int, ws: int):
+        from hybrid_sparse_linear_lightning_b200 import shard
+        ln, sp = w.linear, w.sparse
+        self.w, self.N = w, N
+        self.grp = shard.ShardedGroup(rank, ws, ln.heads, sp.q_heads, sp.kv_heads,
+                                      shard.group_subgroups(ws, sp.kv_heads))
+        lo, hi = self.grp.lin
+        self.lin_inputs = []
+        for l in range(w.n_linear):
+            full = wl.layer_inputs(w, l, dev, seqlen=N)
+            self.lin_inputs.append([t[:, :, lo:hi].contiguous() for t in full])
+            del full
+            torch.cuda.empty_cache()
+        s_ = self.grp.sp
+        full = wl.layer_inputs(w, w.n_linear, dev, seqlen=N)
+        self.sp_inputs = [full[0][:, :, s_.q_lo:s_.q_hi].contiguous(),
+                          full[1][:, :, s_.kv_lo:s_.kv_hi].contiguous(),
+                          full[2][:, :, s_.kv_lo:s_.kv_hi].contiguous(),
+                          full[3][:, :, s_.q_lo:s_.q_hi].contiguous()]
+        del full
+        torch.cuda.empty_cache()
+        self.lam = torch.tensor(wl.lam_schedule(ln)[lo:hi], dtype=torch.float32, device=dev)
+        self.wt = wl.rms_weights(ln.head_dim, dev)
+
+    def step(self, timed_calls=None):
+        w, sp = self.w, self.w.sparse
+        for l in range(w.n_linear):
+            q, k, v, g = self.lin_inputs[l]
+            self.grp.linear(q, k, v, g, self.lam, self.wt, self.wt, chunk=w.linear.chunk)
+        q, k, v, g = self.sp_inputs
+        self.grp.sparse(q, k, v, g, self.wt, self.wt, block=sp.block, topk=sp.topk,
+                        n_init=sp.n_init, n_local=sp.n_local)
+
+
+def run_sharded(args):
+    """Strong scaling: one layer group split by heads over the ranks."""
+    rank, ws, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from hybrid_sparse_linear_lightning_b200 import sala
+    w = wl.WORKLOADS[args.workload]
+    N = args.seqlen or w.seqlen
+    grp = ShardedGroupPrefill(w, N, dev, rank, ws)
+    for _ in range(args.warmup):
+        grp.step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(ws)
+    torch.cuda.synchronize()
+    l0 = sala.sala_kernel_launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        grp.step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+    value = w.batch * N * args.steps / (ms / 1e3)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic N(0,1) inputs, seeded (no trained weights)",
+            "config": dict(config_of(w, N, ws), parallelism=f"heads x{ws}"),
+            "gpu_launches": sala.sala_kernel_launch_count() - l0, "clocks": clk}), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
 
 
 KERNEL_SOURCES = {
@@ -823,6 +907,9 @@ def main():
                     help="oracle samples timed for cpu_baseline (a few seconds each)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing the other layer-group workloads")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="replicas: one independent group per GPU (weak scaling); heads: one "
+                         "group split by heads over the GPUs (strong scaling)")
     ap.add_argument("--decode-steps", type=int, default=256,
                     help="decode tokens timed after a 1M-token prefill (0: skip)")
     args = ap.parse_args()
@@ -830,6 +917,8 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard == "heads":
+        run_sharded(args)
     else:
         run_ours(args)
 

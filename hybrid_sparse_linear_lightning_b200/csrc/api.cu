@@ -162,17 +162,42 @@ sala_status run_linear(const sala_linear_desc* d, const void* q, const void* k, 
   return launch_status();
 }
 
+// Normalisation and block means of the sparse layer: q_norm, k_norm, kbar,
+// and qsum [B, nb, Hkv, D] = sum over the group's q heads of the block-mean
+// normalised queries.
+template <typename T, int D>
+sala_status run_select_begin(const sala_sparse_desc* d, const void* q, const void* k,
+                             const float* wq, const float* wk, void* q_norm, void* k_norm,
+                             float* kbar, float* qsum, cudaStream_t st) {
+  const int nb = d->seqlen / d->block;
+  sparse_prologue_kernel<T, D><<<d->batch * nb * d->kv_heads, kPrologueThreads, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), wq, wk,
+      static_cast<__nv_bfloat16*>(q_norm), static_cast<__nv_bfloat16*>(k_norm), qsum, kbar,
+      d->seqlen, d->q_heads, d->kv_heads, d->block, d->rms_eps);
+  return launch_status();
+}
+
+// Block-mean ranking of every query block from qsum and kbar.
+template <int D>
+sala_status run_select_finish(const sala_sparse_desc* d, const float* qsum, const float* kbar,
+                              int32_t* idx, cudaStream_t st) {
+  const int nb = d->seqlen / d->block;
+  const int width = d->topk + d->n_init + d->n_local;
+  const size_t smem = (size_t)nb * sizeof(uint32_t);
+  if (allow_smem(select_topk_kernel<D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  select_topk_kernel<D><<<d->batch * d->kv_heads * nb, kSelectThreads, smem, st>>>(
+      qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width);
+  return launch_status();
+}
+
 template <typename T, int D>
 sala_status run_select(const sala_sparse_desc* d, const void* q, const void* k, const float* wq,
                        const float* wk, void* q_norm, void* k_norm, float* kbar, int32_t* idx,
                        char* ws, cudaStream_t st) {
   const int nb = d->seqlen / d->block;
   float* qsum = reinterpret_cast<float*>(ws);
-  sparse_prologue_kernel<T, D><<<d->batch * nb * d->kv_heads, kPrologueThreads, 0, st>>>(
-      static_cast<const T*>(q), static_cast<const T*>(k), wq, wk,
-      static_cast<__nv_bfloat16*>(q_norm), static_cast<__nv_bfloat16*>(k_norm), qsum, kbar,
-      d->seqlen, d->q_heads, d->kv_heads, d->block, d->rms_eps);
-  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  if (run_select_begin<T, D>(d, q, k, wq, wk, q_norm, k_norm, kbar, qsum, st) != SALA_OK)
+    return SALA_ERR_CUDA;
   const int width = d->topk + d->n_init + d->n_local;
   if (d->selection == SALA_SELECT_TOKEN_SOFTMAX) {
     const size_t ts_smem = TsLayout<D>::bytes(nb);
@@ -182,11 +207,7 @@ sala_status run_select(const sala_sparse_desc* d, const void* q, const void* k, 
         d->n_local, width, d->rms_eps);
     return launch_status();
   }
-  const size_t smem = (size_t)nb * sizeof(uint32_t);
-  if (allow_smem(select_topk_kernel<D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
-  select_topk_kernel<D><<<d->batch * d->kv_heads * nb, kSelectThreads, smem, st>>>(
-      qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width);
-  return launch_status();
+  return run_select_finish<D>(d, qsum, kbar, idx, st);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -525,6 +546,37 @@ sala_status sala_sparse_select(const sala_sparse_desc* d, const void* q, const v
   if (d->head_dim == 128)
     return run_select<float, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
   return run_select<float, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, idx, ws, st);
+}
+
+sala_status sala_sparse_select_begin(const sala_sparse_desc* d, const void* q, const void* k,
+                                     const float* wq, const float* wk, void* q_norm,
+                                     void* k_norm, float* kbar, float* qsum, void* stream) {
+  sala_status s = check_sparse(d);
+  if (s != SALA_OK) return s;
+  if (d->selection != SALA_SELECT_BLOCK_MEAN) return SALA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(wq) || !aligned16(wk) || !aligned16(q_norm) ||
+      !aligned16(k_norm) || !aligned16(kbar) || !aligned16(qsum))
+    return SALA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == SALA_BF16) {
+    if (d->head_dim == 128)
+      return run_select_begin<__nv_bfloat16, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, qsum, st);
+    return run_select_begin<__nv_bfloat16, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, qsum, st);
+  }
+  if (d->head_dim == 128)
+    return run_select_begin<float, 128>(d, q, k, wq, wk, q_norm, k_norm, kbar, qsum, st);
+  return run_select_begin<float, 64>(d, q, k, wq, wk, q_norm, k_norm, kbar, qsum, st);
+}
+
+sala_status sala_sparse_select_finish(const sala_sparse_desc* d, const float* qsum,
+                                      const float* kbar, int32_t* idx, void* stream) {
+  sala_status s = check_sparse(d);
+  if (s != SALA_OK) return s;
+  if (d->selection != SALA_SELECT_BLOCK_MEAN) return SALA_ERR_UNSUPPORTED;
+  if (!aligned16(qsum) || !aligned16(kbar) || !aligned16(idx)) return SALA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->head_dim == 128) return run_select_finish<128>(d, qsum, kbar, idx, st);
+  return run_select_finish<64>(d, qsum, kbar, idx, st);
 }
 
 sala_status sala_sparse_prefill(const sala_sparse_desc* d, const void* q_norm,

@@ -36,6 +36,7 @@ EXPORTED = [
     "sala_decode_workspace_size", "sala_decode_step", "sala_status_string",
     "sala_get_device_status", "sala_version", "sala_kernel_launch_count",
     "sala_sparse_select_noalloc", "sala_selftest_bounded_wait",
+    "sala_sparse_select_begin", "sala_sparse_select_finish",
 ]
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -97,6 +98,8 @@ def _load():
         "sala_kernel_launch_count": (ctypes.c_uint64, []),
         "sala_sparse_select_noalloc": (I, [P] + [P] * 8 + [P]),
         "sala_selftest_bounded_wait": (I, [P]),
+        "sala_sparse_select_begin": (I, [P] + [P] * 8 + [P]),
+        "sala_sparse_select_finish": (I, [P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -192,6 +195,18 @@ def sala_sparse_select_noalloc(d: SparseDesc, q, k, wq, wk, q_norm, k_norm, kbar
     return LIB.sala_sparse_select_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
                                           _ptr(q_norm), _ptr(k_norm), _ptr(kbar), _ptr(idx),
                                           _stream(stream))
+
+
+def sala_sparse_select_begin(d: SparseDesc, q, k, wq, wk, q_norm, k_norm, kbar, qsum,
+                             stream=None) -> int:
+    return LIB.sala_sparse_select_begin(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(wq), _ptr(wk),
+                                        _ptr(q_norm), _ptr(k_norm), _ptr(kbar), _ptr(qsum),
+                                        _stream(stream))
+
+
+def sala_sparse_select_finish(d: SparseDesc, qsum, kbar, idx, stream=None) -> int:
+    return LIB.sala_sparse_select_finish(ctypes.byref(d), _ptr(qsum), _ptr(kbar), _ptr(idx),
+                                         _stream(stream))
 
 
 def sala_sparse_prefill(d: SparseDesc, q_norm, k_norm, v, gate, idx, out, workspace=None,

@@ -134,6 +134,23 @@ sala_status sala_sparse_select(const sala_sparse_desc* d, const void* q, const v
                                float* kbar, int32_t* idx, void* workspace, size_t ws_bytes,
                                void* stream);
 
+/* Split form of sala_sparse_select, for a kv group whose q heads are spread
+ * over several callers (head-sharded prefill on several GPUs).
+ * sala_sparse_select_begin normalises and writes q_norm, k_norm and kbar as
+ * sala_sparse_select does, plus qsum [B, N/block, Hkv, d] fp32: for each kv
+ * head, the sum over THIS call's q heads of the block-mean normalised
+ * queries.  The callers that share a kv group add their qsum (an
+ * all-reduce), and each calls sala_sparse_select_finish with the total; it
+ * ranks every query block by <qsum_b, kbar_j> / sqrt(d) and writes idx
+ * exactly as sala_sparse_select does (SALA_SELECT_BLOCK_MEAN only; other
+ * rules return SALA_ERR_UNSUPPORTED).  No workspace: qsum is the caller's.
+ * Called back to back with one caller, the pair equals sala_sparse_select. */
+sala_status sala_sparse_select_begin(const sala_sparse_desc* d, const void* q, const void* k,
+                                     const float* wq, const float* wk, void* q_norm,
+                                     void* k_norm, float* kbar, float* qsum, void* stream);
+sala_status sala_sparse_select_finish(const sala_sparse_desc* d, const float* qsum,
+                                      const float* kbar, int32_t* idx, void* stream);
+
 /* Allocation-free variant of sala_sparse_select (no counterpart on the
  * pages: it exists for callers, not for the method).  Same arguments and
  * results, minus the workspace: its scratch is a fixed array of

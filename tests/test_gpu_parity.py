@@ -389,3 +389,51 @@ def test_sparse_token_softmax_selection(sala, name, seqlen):
     assert n_tie <= max(1, gidx.shape[1] * gidx.shape[2] // 50), n_tie
     want = oracle.sigmoid(f64(g)) * oracle.sparse_attention(qh, kh, f64(v), gidx, sp.block)
     assert rel_err(f64(out), want) <= TOL
+
+
+def test_split_selection_virtual_shards(sala):
+    """The q heads of each kv group split in two halves, as two ranks of a
+    head-sharded run hold them: sala_sparse_select_begin on each half, the
+    two block-mean query sums added (what the ranks' all-reduce does),
+    sala_sparse_select_finish, attention per half.  The assembled layer
+    matches the oracle (indices within the tie window, outputs over the
+    GPU's own lists)."""
+    from hybrid_sparse_linear_lightning_b200 import shard
+    dev = torch.device("cuda")
+    w = _w("group_32k")
+    sp = w.sparse
+    N = 4160
+    q, k, v, g = wl.layer_inputs(w, w.n_linear, dev, seqlen=N)
+    wt = wl.rms_weights(128, dev)
+    be = shard.LibsalaBackend()
+    G = sp.q_heads // sp.kv_heads
+    half = G // 2
+    out = torch.empty_like(g)
+    idx_all = []
+    for gg in range(sp.kv_heads):
+        kk = k[:, :, gg:gg + 1].contiguous()
+        vv = v[:, :, gg:gg + 1].contiguous()
+        sels = []
+        for hh in range(2):
+            lo = gg * G + hh * half
+            sels.append((lo, be.select_begin(q[:, :, lo:lo + half].contiguous(), kk, wt, wt,
+                                             block=64, topk=sp.topk, n_init=sp.n_init,
+                                             n_local=sp.n_local)))
+        total = sels[0][1]["qsum"] + sels[1][1]["qsum"]
+        for _, s_ in sels:
+            s_["qsum"].copy_(total)
+        idx = be.select_finish(sels[0][1])
+        assert torch.equal(idx, be.select_finish(sels[1][1]))
+        for lo, s_ in sels:
+            out[:, :, lo:lo + half] = be.sparse_prefill(s_, vv, g[:, :, lo:lo + half].contiguous(),
+                                                        idx)
+        idx_all.append(idx)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    gidx = torch.cat(idx_all, dim=1).cpu().numpy()
+    _, (qh, kh, _, ridx, scores) = oracle.sparse_layer(
+        f64(q), f64(k), f64(v), f64(g), f64(wt), f64(wt), block=64, topk=sp.topk,
+        n_init=sp.n_init, n_local=sp.n_local)
+    check_index_rows(gidx, ridx, scores, sp.topk, sp.n_init, sp.n_local)
+    want = oracle.sigmoid(f64(g)) * oracle.sparse_attention(qh, kh, f64(v), gidx, 64)
+    assert rel_err(f64(out), want) <= TOL
