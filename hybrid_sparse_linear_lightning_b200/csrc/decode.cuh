@@ -55,16 +55,18 @@ constexpr int kDecMaxLayers = 8;
 
 // Control words at the start of the workspace (zeroed by the host before
 // each launch), each on its own 128-byte line: the barriers' arrival counts
-// and release flags, and per (batch, kv head) the number of scored chunks.
+// and release flags, the P0 work counter, and per (batch, kv head) the
+// number of scored chunks.
 constexpr int kDecCtlBarriers = 2;
 constexpr int kDecLine = 32;            // words per 128-byte line
-__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (2 * kDecCtlBarriers + bg); }
+__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (2 * kDecCtlBarriers + 1 + bg); }
 __device__ __forceinline__ unsigned* dec_bar_count(unsigned* ctl, int i) { return ctl + kDecLine * i; }
 __device__ __forceinline__ unsigned* dec_bar_flag(unsigned* ctl, int i) {
   return ctl + kDecLine * (kDecCtlBarriers + i);
 }
+__device__ __forceinline__ unsigned* dec_work(unsigned* ctl) { return ctl + kDecLine * 2 * kDecCtlBarriers; }
 __device__ __forceinline__ unsigned* dec_bg_done(unsigned* ctl, int bg) {
-  return ctl + kDecLine * (2 * kDecCtlBarriers + bg);
+  return ctl + kDecLine * (2 * kDecCtlBarriers + 1 + bg);
 }
 
 struct DecodeParams {
@@ -439,16 +441,27 @@ __device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem
   }
   // 2. above / boundary lists (slot order is arbitrary; the result is not)
   const unsigned T = (unsigned)s_T;
-  for (int c = tid; c < p.n_cand; c += kDecThreads) {
-    const uint32_t key = __ldcg(p.keys + (long long)bg * p.capb + c);
-    const unsigned bin = key >> (32 - kDecBinBits);
-    if (bin > T) {
-      const int slot = atomicAdd(&s_n_above, 1);
-      if (slot < p.topk) chosen[slot] = c;
-      else set_status(kStatusBounds);
-    } else if (bin == T) {
-      const int slot = atomicAdd(&s_n_bnd, 1);
-      if (slot < kDecBndMax) sb[slot] = make_uint2(key, (unsigned)c);
+  constexpr int kBatch = 16;            // keys in flight per thread
+  for (int c0 = 0; c0 < p.n_cand; c0 += kBatch * kDecThreads) {
+    uint32_t kv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + u * kDecThreads + tid;
+      kv[u] = c < p.n_cand ? __ldcg(p.keys + (long long)bg * p.capb + c) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + u * kDecThreads + tid;
+      if (c >= p.n_cand) continue;
+      const unsigned bin = kv[u] >> (32 - kDecBinBits);
+      if (bin > T) {
+        const int slot = atomicAdd(&s_n_above, 1);
+        if (slot < p.topk) chosen[slot] = c;
+        else set_status(kStatusBounds);
+      } else if (bin == T) {
+        const int slot = atomicAdd(&s_n_bnd, 1);
+        if (slot < kDecBndMax) sb[slot] = make_uint2(kv[u], (unsigned)c);
+      }
     }
   }
   __syncthreads();
@@ -531,21 +544,43 @@ __device__ void dec_attn_unit(const DecodeParams& p, int u, unsigned char* smem_
   }
   const long long kend = min((long long)(j + 1) * p.BLK, p.pos + 1);
   const int nk = (int)(kend - (long long)j * p.BLK);
-  for (int e = tid; e < 64 * NC; e += kDecThreads) {
-    const int sr = e / NC, c = e % NC;
-    uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
-    if (sr < nk) {
-      const long long off = (((long long)b * p.cap + (long long)j * p.BLK + sr) * p.Hkv + g) * D + 8 * c;
-      kv = __ldcg(reinterpret_cast<const uint4*>(p.k_cache + off));
-      vv = __ldcg(reinterpret_cast<const uint4*>(p.v_cache + off));
-    }
-    ks[sr * NC + (c ^ (sr & (NC - 1)))] = kv;
-    vs[sr * NC + (c ^ (sr & (NC - 1)))] = vv;
-  }
   {
+    // every load of the unit is issued before the first shared-memory store
+    constexpr int PER = (64 * NC + kDecThreads - 1) / kDecThreads;
+    constexpr int QPER = 1;     // one query float4 per thread in flight (G * D / 4 <= 512 at G = 16)
+    uint4 kv[PER], vv[PER];
+    float4 qv[QPER];
     const float4* qsrc = reinterpret_cast<const float4*>(p.qhat + ((long long)b * p.Hq + g * G) * D);
-    float4* qdst = reinterpret_cast<float4*>(qs);
-    for (int e = tid; e < G * D / 4; e += kDecThreads) qdst[e] = __ldcg(qsrc + e);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = tid + u * kDecThreads, sr = e / NC, c = e % NC;
+      kv[u] = vv[u] = make_uint4(0, 0, 0, 0);
+      if (e < 64 * NC && sr < nk) {
+        const long long off = (((long long)b * p.cap + (long long)j * p.BLK + sr) * p.Hkv + g) * D + 8 * c;
+        kv[u] = __ldcg(reinterpret_cast<const uint4*>(p.k_cache + off));
+        vv[u] = __ldcg(reinterpret_cast<const uint4*>(p.v_cache + off));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < QPER; ++u) {
+      const int e = tid + u * kDecThreads;
+      if (e < G * D / 4) qv[u] = __ldcg(qsrc + e);
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int e = tid + u * kDecThreads, sr = e / NC, c = e % NC;
+      if (e < 64 * NC) {
+        ks[sr * NC + (c ^ (sr & (NC - 1)))] = kv[u];
+        vs[sr * NC + (c ^ (sr & (NC - 1)))] = vv[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < QPER; ++u) {
+      const int e = tid + u * kDecThreads;
+      if (e < G * D / 4) reinterpret_cast<float4*>(qs)[e] = qv[u];
+    }
+    for (int e = tid + QPER * kDecThreads; e < G * D / 4; e += kDecThreads)
+      reinterpret_cast<float4*>(qs)[e] = __ldcg(qsrc + e);
   }
   __syncthreads();
   // logits: thread (key sr, heads hq0 + 8 m)
@@ -608,32 +643,59 @@ template <typename T, int D>
 __device__ void dec_combine_unit(const DecodeParams& p, int u, float* sm) {
   constexpr int DP = D + 4;
   constexpr int NQ = kDecThreads / D;
+  constexpr int kBatch = 18;             // partials in flight per thread
   const int hq = u % p.Hq, b = u / p.Hq;
   const int G = p.Hq / p.Hkv, g = hq / G, h = hq % G;
   const int tid = threadIdx.x;
-  float* wts = sm;                       // [width]
-  float* red = sm + p.width;             // [NQ][D]
+  float* wts = sm;                       // [width] weights, then [width] sums
+  float* lsum = sm + p.width;
+  float* red = sm + 2 * p.width;         // [NQ][D]
   __shared__ float s_l;
   const float* pb = p.part + (((long long)b * p.Hkv + g) * p.width * G + h) * DP;
   const long long pstride = (long long)G * DP;
+  const int col = tid % D, qtr = tid / D;
+  float o = 0.f;
+  // this thread's first batch of partial columns is loaded before the weights
+  // are formed (every thread runs this block: it holds the CTA barriers)
+  float pv[kBatch];
+#pragma unroll
+  for (int v = 0; v < kBatch; ++v) {
+    const int e = qtr + v * NQ;
+    pv[v] = e < p.width ? __ldcg(pb + e * pstride + 4 + col) : 0.f;
+  }
+  for (int e = tid; e < p.width; e += kDecThreads) {
+    wts[e] = __ldcg(pb + e * pstride);
+    lsum[e] = __ldcg(pb + e * pstride + 1);
+  }
+  __syncthreads();
   if (tid < 32) {
     float M = -INFINITY;
-    for (int e = tid; e < p.width; e += 32) M = fmaxf(M, __ldcg(pb + e * pstride));
+    for (int e = tid; e < p.width; e += 32) M = fmaxf(M, wts[e]);
     M = warp_max(M);
     float L = 0.f;
     for (int e = tid; e < p.width; e += 32) {
-      const float m = __ldcg(pb + e * pstride);
+      const float m = wts[e];
       const float f = m == -INFINITY ? 0.f : exp2f(m - M);
-      L = fmaf(f, __ldcg(pb + e * pstride + 1), L);
+      L = fmaf(f, lsum[e], L);
       wts[e] = f;
     }
     L = warp_sum(L);
     if (tid == 0) s_l = L;
   }
   __syncthreads();
-  const int col = tid % D, qtr = tid / D;
-  float o = 0.f;
-  for (int e = qtr; e < p.width; e += NQ) o = fmaf(wts[e], __ldcg(pb + e * pstride + 4 + col), o);
+  for (int e0 = qtr;; e0 += kBatch * NQ) {
+#pragma unroll
+    for (int v = 0; v < kBatch; ++v) {
+      const int e = e0 + v * NQ;
+      if (e < p.width) o = fmaf(wts[e], pv[v], o);
+    }
+    if (e0 + kBatch * NQ >= p.width) break;
+#pragma unroll
+    for (int v = 0; v < kBatch; ++v) {
+      const int e = e0 + kBatch * NQ + v * NQ;
+      pv[v] = e < p.width ? __ldcg(pb + e * pstride + 4 + col) : 0.f;
+    }
+  }
   red[qtr * D + col] = o;
   __syncthreads();
   if (tid < D) {
@@ -660,13 +722,26 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
 
   // P0: scores + histogram (+ selection by the last chunk of each (b, g)),
   // linear layers, sparse prep; direct index rows when nothing ranks
+  // Units are handed out by a work counter in order (scores first, so that
+  // the selections start early), each CTA asking for its next unit while it
+  // works on the current one.
   const int n_direct = ranked ? 0 : BG;
-  for (int u = blockIdx.x; u < n_score + n_lin + p.B + n_direct; u += gridDim.x) {
+  const int n_p0 = n_score + n_lin + p.B + n_direct;
+  __shared__ int s_unit;
+  if (threadIdx.x == 0) s_unit = (int)atomicAdd(dec_work(p.ctl), 1u);
+  __syncthreads();
+  int u = s_unit;
+  while (u < n_p0) {
+    unsigned nxt = 0;
+    if (threadIdx.x == 0) nxt = atomicAdd(dec_work(p.ctl), 1u);
     if (u < n_score) dec_score_unit<T, D>(p, u, sm);
     else if (u < n_score + n_lin) dec_linear_unit<T, D>(p, u - n_score, sm);
     else if (u < n_score + n_lin + p.B) dec_sparse_prep_unit<T, D>(p, u - n_score - n_lin);
     else dec_direct_row(p, u - n_score - n_lin - p.B);
     __syncthreads();
+    if (threadIdx.x == 0) s_unit = (int)nxt;
+    __syncthreads();
+    u = s_unit;
   }
   if (!dec_grid_sync(dec_bar_count(p.ctl, 0), dec_bar_flag(p.ctl, 0), [] {})) return;
   // P1: attention partials
@@ -690,7 +765,7 @@ inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int widt
                       (size_t)2 * G * D * 4 + (size_t)G * 8;
   const size_t resolve = (size_t)2 * topk * 4 + 16 +
                          std::max((size_t)kDecBndMax * 8, (size_t)capb * 4);   // dec_select_bg
-  const size_t comb = (size_t)width * 4 + (size_t)(kDecThreads / D) * D * 4;
+  const size_t comb = (size_t)2 * width * 4 + (size_t)(kDecThreads / D) * D * 4;
   return std::max(std::max(std::max(score, lin), std::max(attn, resolve)), comb);
 }
 

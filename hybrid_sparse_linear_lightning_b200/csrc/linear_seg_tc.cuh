@@ -81,14 +81,20 @@ struct RopeF32 {
   float th[64];
 };
 
+// Frequencies theta_l and theta_{l+32} (fp64) of lane l of the calling warp,
+// read once per kernel and kept in registers.
+__device__ __forceinline__ double2 rope_lane_freqs(const RopeFreq& rf) {
+  const int lane = threadIdx.x & 31;
+  return make_double2(rf.inv[lane], rf.inv[lane + 32]);
+}
+
 // Base angles of a tile that starts at position p: lane l of the calling warp
 // returns (p * theta_l, p * theta_{l+32}) reduced modulo 2 pi, formed in fp64
 // (|p| < 2^53) and rounded to fp32.
-__device__ __forceinline__ float2 rope_tile_base(long long p, const RopeFreq& rf) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ float2 rope_tile_base(long long p, double2 th) {
   constexpr double kTwoPi = 6.283185307179586476925286766559;
   constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-  const double a = (double)p * rf.inv[lane], b = (double)p * rf.inv[lane + 32];
+  const double a = (double)p * th.x, b = (double)p * th.y;
   return make_float2((float)fma(-rint(a * kInvTwoPi), kTwoPi, a),
                      (float)fma(-rint(b * kInvTwoPi), kTwoPi, b));
 }
@@ -267,19 +273,23 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int a = (warp - 4) >> 2;
+    const double2 th = rope_lane_freqs(rf);
     bool ok = true;
     for (int c = a; ok && c < nt; c += kLsSumStages) {
       const int st = a;
       const int tile_start = (t0 + c) * kLsTile;
       const int Lt = min(kLsTile, N - tile_start);
+      // k^_j (normalised, rotated at its position) scaled by
+      // lam^(seg_end - 1 - j) = lam^(seg_end - tile_end) lam^(L - 1 - r); the
+      // tile factor is formed in fp64 by one lane while the loads land
+      float ft = 0.f;
+      if (lane == 0) ft = (float)pow((double)lam, (double)(seg_end - (tile_start + Lt)));
+      ft = __shfl_sync(0xffffffffu, ft, 0);
+      const float2 base = rope_tile_base(pos0 + tile_start, th);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + st, (c / kLsSumStages) & 1));
       if (!ok) break;
-      // k^_j (normalised, rotated at its position) scaled by
-      // lam^(seg_end - 1 - j) = lam^(seg_end - tile_end) lam^(L - 1 - r)
-      const float ft = (float)pow((double)lam, (double)(seg_end - (tile_start + Lt)));
       const float f = r < Lt ? ft * pw[Lt - 1 - r] : 0.f;
-      sw128_norm_rope_row(smem + st * L::kStage, r, wsm, eps, rope_tile_base(pos0 + tile_start, rf),
-                          rt, f);
+      sw128_norm_rope_row(smem + st * L::kStage, r, wsm, eps, base, rt, f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(k_ready + st);
@@ -560,11 +570,12 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const double2 th = rope_lane_freqs(rf);
     for (int c = 0; c < nt; ++c) {
       // raw q row -> q^ (RMSNorm, RoPE at its position), in place
+      const float2 base = rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, th);
       if (!__all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1))) break;
-      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wsm, eps,
-                          rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, rf), rt, 1.f);
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wsm, eps, base, rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qk_ready);
@@ -643,13 +654,14 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       }
     }
     bool ok = true;
+    const double2 th = rope_lane_freqs(rf);
     for (int c = 0; ok && c < nt; ++c) {
       const int Lt = tile_len(c);
       // raw k row -> k^ (RMSNorm, RoPE at its position), in place
+      const float2 base = rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, th);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1));
       if (!ok) break;
-      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wsm + D, eps,
-                          rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, rf), rt, 1.f);
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wsm + D, eps, base, rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qk_ready);
