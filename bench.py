@@ -580,6 +580,70 @@ def time_selection_variant(w: wl.Workload, dev, sala, steps: int = 5, warmup: in
             "peak_source": "fp32 FMA lanes x SMs x max clock (no measured fp32 peak)"}
 
 
+BLOCK_HIDDEN, BLOCK_FFN = 4096, 16384     # synthetic decoder-block widths (pages give none)
+
+
+def block_group_gemm_flops(w: wl.Workload, N: int, hidden=BLOCK_HIDDEN, ffn=BLOCK_FFN) -> float:
+    """Dense GEMM work of one group of decoder blocks: q, k, v, gate and
+    output projections and the SwiGLU FFN (2 FLOP per multiply-add)."""
+    ln, sp = w.linear, w.sparse
+    d = ln.head_dim
+    lin = 2 * hidden * (2 * ln.heads * d + 2 * ln.heads * d) + 2 * ln.heads * d * hidden
+    spa = 2 * hidden * (2 * sp.q_heads * d + 2 * sp.kv_heads * d) + 2 * sp.q_heads * d * hidden
+    ffn_f = 2 * hidden * 2 * ffn + 2 * ffn * hidden
+    return float(w.batch * N) * (w.n_linear * (lin + ffn_f) + spa + ffn_f)
+
+
+def time_block_group(w: wl.Workload, N: int, dev, sala, peaks, steps=3, warmup=2):
+    """A layer group of full decoder blocks (sala_block_prefill x 4) on a
+    residual stream x [1, N, 4096] fp32, synthetic weights; CUDA events."""
+    ln, sp = w.linear, w.sparse
+    d = ln.head_dim
+    hidden = ln.heads * d
+    gen = torch.Generator(device=dev).manual_seed(w.seed)
+    bufs = [torch.randn((w.batch, N, hidden), generator=gen, device=dev), None]
+    bufs[1] = torch.empty_like(bufs[0])
+    bd = sala.BlockDesc(hidden, BLOCK_FFN, 1e-6)
+    ld = sala.linear_desc(w.batch, N, ln.heads, d, ln.chunk, w.torch_dtype)
+    sd = sala.sparse_desc(w.batch, N, sp.q_heads, sp.kv_heads, d, sp.block, sp.topk, sp.n_init,
+                          sp.n_local, w.torch_dtype)
+    layers = []
+    for l in range(w.n_linear + 1):
+        kind_lin = l < w.n_linear
+        wt = wl.block_weights(hidden, BLOCK_FFN, ln.heads if kind_lin else sp.q_heads,
+                              ln.heads if kind_lin else sp.kv_heads, d, l, dev, seed=w.seed)
+        layers.append((ld if kind_lin else None, None if kind_lin else sd, wt, sala.block_weights(wt)))
+    ws = sala.workspace(max(sala.sala_block_workspace_size(bd, a, b) for a, b, _, _ in layers), dev)
+    lam = torch.tensor(wl.lam_schedule(ln), dtype=torch.float32, device=dev)
+
+    def step():
+        for l, (a, b, _, bw) in enumerate(layers):
+            st = sala.sala_block_prefill(bd, a, b, bw, lam if a is not None else None,
+                                         bufs[l % 2], bufs[(l + 1) % 2], None, ws)
+            if st != 0:
+                raise RuntimeError("sala_block_prefill: " + sala.status_string(st))
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if sala.sala_get_device_status() != 0:
+        raise RuntimeError("device status word set in the block group")
+    ms = e0.elapsed_time(e1) / steps
+    gemm = block_group_gemm_flops(w, N) / (ms / 1e3) / 1e12
+    return {"workload": w.name, "seq_len": N, "hidden": hidden, "ffn": BLOCK_FFN,
+            "ms_per_step": round(ms, 3), "tokens_per_s": round(w.batch * N / (ms / 1e3), 1),
+            "gemm_tflops_over_step": round(gemm, 1),
+            "gemm_frac_of_burst_bf16": round(gemm / peaks["bf16_tflops"], 4),
+            "note": "3 linear + 1 sparse decoder blocks, synthetic weights; GEMMs in cuBLASLt"}
+
+
 def run_ours(args):
     rank, ws, local = dist_setup()
     dev = torch.device("cuda", local)
@@ -629,6 +693,14 @@ def run_ours(args):
         variants = [time_selection_variant(wl.WORKLOADS["group_32k"], dev, sala)]
         torch.cuda.empty_cache()
 
+    blocks = None
+    if not args.no_blocks:
+        blocks = []
+        for name in ("group_32k", "group_256k"):
+            blocks.append(time_block_group(wl.WORKLOADS[name], wl.WORKLOADS[name].seqlen, dev,
+                                           sala, peaks))
+            torch.cuda.empty_cache()
+
     dec = None
     if args.decode_steps > 0:
         dec = run_decode(wl.WORKLOADS["group_1m"], args.decode_steps, dev, sala, peaks, ws)
@@ -656,7 +728,8 @@ def run_ours(args):
             "tensor_frac_of_step": round(sparse_attn_flops(w, N) / (ms_per_step / 1e3) / 1e12
                                          / peaks["bf16_tflops"], 4),
             "e2e": e2e, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu,
-            "per_config": per_config, "selection_variants": variants, "decode": dec,
+            "per_config": per_config, "selection_variants": variants, "blocks": blocks,
+            "decode": dec,
         }
         print(json.dumps(out), flush=True)
     if ws > 1:
@@ -907,6 +980,8 @@ def main():
                     help="oracle samples timed for cpu_baseline (a few seconds each)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing the other layer-group workloads")
+    ap.add_argument("--no-blocks", action="store_true",
+                    help="skip timing the full decoder-block groups")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="replicas: one independent group per GPU (weak scaling); heads: one "
                          "group split by heads over the GPUs (strong scaling)")

@@ -18,6 +18,8 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
     "--expt-relaxed-constexpr",
+    # the decoder block's GEMMs
+    "-lcublasLt", "-Xlinker", "-rpath,/usr/local/cuda/lib64",
 ]
 
 

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include "../../include/sala.h"
+#include "block.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "linear_simt.cuh"
@@ -22,6 +23,7 @@
 #include "sparse_simt.cuh"
 #include "sparse_tc.cuh"
 
+#include <cublasLt.h>
 #include <cudaTypedefs.h>
 
 using namespace sala;
@@ -484,6 +486,168 @@ sala_status noalloc_scratch(void** out) {
   return SALA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Decoder block around the attention: GEMMs in cuBLASLt.
+
+// One cuBLASLt handle per device, created on first use with that device
+// current (host-side object; it allocates no device memory).
+cublasLtHandle_t lt_handle() {
+  static std::mutex mu;
+  static cublasLtHandle_t handles[kMaxDevices] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!handles[dev] && cublasLtCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
+  return handles[dev];
+}
+
+constexpr size_t kLtWorkspace = (size_t)32 << 20;
+
+// D[m, o] = alpha * sum_k X[m, k] W[o, k] + beta * C[m, o]   (X, W bf16 row
+// major; C, D of type `cd`, row major; fp32 accumulation).  In cuBLASLt's
+// column-major terms: D^T [out, rows] = op_T(W^T [in, out]) * X^T [in, rows].
+sala_status lt_gemm(cudaStream_t st, const void* W, const void* X, const void* C, void* D,
+                    long long rows, int in, int out, cudaDataType_t cd, float beta, void* lt_ws) {
+  cublasLtHandle_t h = lt_handle();
+  if (!h) return SALA_ERR_CUDA;
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  sala_status res = SALA_ERR_CUDA;
+  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
+  const float alpha = 1.0f;
+  size_t ws_bytes = kLtWorkspace;
+  cublasLtMatmulHeuristicResult_t heur;
+  int found = 0;
+  if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) goto done;
+  if (cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)) ||
+      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)))
+    goto done;
+  if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, in, out, in) ||
+      cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, in, rows, in) ||
+      cublasLtMatrixLayoutCreate(&lc, cd, out, rows, out))
+    goto done;
+  if (cublasLtMatmulPreferenceCreate(&pref) ||
+      cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
+                                           &ws_bytes, sizeof(ws_bytes)))
+    goto done;
+  if (cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &heur, &found) ||
+      found < 1)
+    goto done;
+  if (cublasLtMatmul(h, op, &alpha, W, la, X, lb, &beta, C ? C : D, lc, D, lc, &heur.algo, lt_ws,
+                     kLtWorkspace, st) == CUBLAS_STATUS_SUCCESS)
+    res = SALA_OK;
+done:
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return res;
+}
+
+struct BlockWs {
+  size_t xn, q, k, v, g, a, u, s, lt, att, total;
+  int hq, hk, d;
+  long long rows;
+};
+
+sala_status check_block(const sala_block_desc* b, const sala_linear_desc* lin,
+                        const sala_sparse_desc* sp, BlockWs* w) {
+  if (!b || (!lin) == (!sp)) return SALA_ERR_INVALID_ARG;
+  if (b->hidden < 8 || b->hidden % 8 || b->ffn < 8 || b->ffn % 8 || !(b->rms_eps >= 0.f))
+    return SALA_ERR_INVALID_ARG;
+  sala_status s = lin ? check_linear(lin) : check_sparse(sp);
+  if (s != SALA_OK) return s;
+  if ((lin ? lin->dtype : sp->dtype) != SALA_BF16) return SALA_ERR_UNSUPPORTED;
+  w->d = lin ? lin->head_dim : sp->head_dim;
+  w->hq = lin ? lin->heads : sp->q_heads;
+  w->hk = lin ? lin->heads : sp->kv_heads;
+  if (w->hq * w->d != b->hidden) return SALA_ERR_INVALID_ARG;
+  w->rows = (long long)(lin ? lin->batch : sp->batch) * (lin ? lin->seqlen : sp->seqlen);
+  const size_t R = (size_t)w->rows;
+  w->xn = 0;
+  w->q = w->xn + align_up(R * b->hidden * 2);
+  w->k = w->q + align_up(R * w->hq * w->d * 2);
+  w->v = w->k + align_up(R * w->hk * w->d * 2);
+  w->g = w->v + align_up(R * w->hk * w->d * 2);
+  w->a = w->g + align_up(R * w->hq * w->d * 2);
+  w->u = w->a + align_up(R * w->hq * w->d * 2);
+  w->s = w->u + align_up(R * 2 * (size_t)b->ffn * 2);
+  w->lt = w->s + align_up(R * (size_t)b->ffn * 2);
+  w->att = w->lt + align_up(kLtWorkspace);
+  if (lin) {
+    w->total = w->att + align_up(linear_ws(lin).total);
+  } else {
+    const size_t nb = (size_t)sp->batch * (sp->seqlen / sp->block);
+    const size_t sel = align_up(nb * sp->kv_heads * sp->head_dim * 4);          // qsum
+    const size_t qn = align_up(R * sp->q_heads * sp->head_dim * 2);
+    const size_t kn = align_up(R * sp->kv_heads * sp->head_dim * 2);
+    const size_t kb = align_up(nb * sp->kv_heads * sp->head_dim * 4);
+    const size_t ix = align_up(nb * sp->kv_heads * (sp->topk + sp->n_init + sp->n_local) * 4);
+    w->total = w->att + sel + qn + kn + kb + ix;
+  }
+  return SALA_OK;
+}
+
+template <int D>
+sala_status run_block(const sala_block_desc* b, const sala_linear_desc* lin,
+                      const sala_sparse_desc* sp, const sala_block_weights* wt,
+                      const float* lambda, const float* x, float* y, float* state_out, char* ws,
+                      const BlockWs& w, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const long long R = w.rows;
+  const int H = b->hidden;
+  bf* xn = reinterpret_cast<bf*>(ws + w.xn);
+  void* q = ws + w.q;
+  void* k = ws + w.k;
+  void* v = ws + w.v;
+  void* g = ws + w.g;
+  void* a = ws + w.a;
+  void* lt = ws + w.lt;
+  // attention sub-block
+  block_rmsnorm_kernel<<<(unsigned)R, kBlkNormThreads, 0, st>>>(x, wt->norm_attn, xn, H, b->rms_eps);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  if (lt_gemm(st, wt->wq, xn, nullptr, q, R, H, w.hq * D, CUDA_R_16BF, 0.f, lt) ||
+      lt_gemm(st, wt->wk, xn, nullptr, k, R, H, w.hk * D, CUDA_R_16BF, 0.f, lt) ||
+      lt_gemm(st, wt->wv, xn, nullptr, v, R, H, w.hk * D, CUDA_R_16BF, 0.f, lt) ||
+      lt_gemm(st, wt->wg, xn, nullptr, g, R, H, w.hq * D, CUDA_R_16BF, 0.f, lt))
+    return SALA_ERR_CUDA;
+  sala_status s;
+  char* att = ws + w.att;
+  if (lin) {
+    s = run_linear<bf, D>(lin, q, k, v, g, lambda, wt->qk_norm_q, wt->qk_norm_k, nullptr,
+                          state_out, a, att, st);
+  } else {
+    const size_t nb = (size_t)sp->batch * (sp->seqlen / sp->block);
+    char* qsum = att;
+    char* qn = qsum + align_up(nb * sp->kv_heads * D * 4);
+    char* kn = qn + align_up((size_t)R * sp->q_heads * D * 2);
+    char* kb = kn + align_up((size_t)R * sp->kv_heads * D * 2);
+    char* ix = kb + align_up(nb * sp->kv_heads * D * 4);
+    s = run_select<bf, D>(sp, q, k, wt->qk_norm_q, wt->qk_norm_k, qn, kn,
+                          reinterpret_cast<float*>(kb), reinterpret_cast<int32_t*>(ix), qsum, st);
+    if (s == SALA_OK)
+      s = run_sparse_prefill<bf, D>(sp, qn, kn, v, g, reinterpret_cast<int32_t*>(ix), a, st);
+  }
+  if (s != SALA_OK) return s;
+  // h = x + a Wo^T (fp32 residual stream, in y)
+  if (lt_gemm(st, wt->wo, a, x, y, R, w.hq * D, H, CUDA_R_32F, 1.f, lt)) return SALA_ERR_CUDA;
+  // feed-forward sub-block
+  block_rmsnorm_kernel<<<(unsigned)R, kBlkNormThreads, 0, st>>>(y, wt->norm_ffn, xn, H, b->rms_eps);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  void* u = ws + w.u;
+  bf* sg = reinterpret_cast<bf*>(ws + w.s);
+  if (lt_gemm(st, wt->w13, xn, nullptr, u, R, H, 2 * b->ffn, CUDA_R_16BF, 0.f, lt))
+    return SALA_ERR_CUDA;
+  const long long n8 = R * (b->ffn / 8);
+  block_swiglu_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(static_cast<const bf*>(u), sg, R,
+                                                                     b->ffn);
+  if (launch_status() != SALA_OK) return SALA_ERR_CUDA;
+  if (lt_gemm(st, wt->w2, sg, y, y, R, b->ffn, H, CUDA_R_32F, 1.f, lt)) return SALA_ERR_CUDA;
+  return SALA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -659,6 +823,33 @@ sala_status sala_decode_step(const sala_decode_desc* d, const sala_decode_io* io
   }
   if (dl == 128) return run_decode<float, 128>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
   return run_decode<float, 64>(d, io, k_cache, v_cache, kbar, ksum, cur_len, ws, st);
+}
+
+size_t sala_block_workspace_size(const sala_block_desc* b, const sala_linear_desc* lin,
+                                 const sala_sparse_desc* sp) {
+  BlockWs w;
+  if (check_block(b, lin, sp, &w) != SALA_OK) return 0;
+  return w.total;
+}
+
+sala_status sala_block_prefill(const sala_block_desc* b, const sala_linear_desc* lin,
+                               const sala_sparse_desc* sp, const sala_block_weights* wt,
+                               const float* lambda, const float* x, float* y, float* state_out,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  BlockWs w;
+  sala_status s = check_block(b, lin, sp, &w);
+  if (s != SALA_OK) return s;
+  if (!wt || !aligned16(x) || !aligned16(y) || x == y || !aligned16(wt->norm_attn) ||
+      !aligned16(wt->wq) || !aligned16(wt->wk) || !aligned16(wt->wv) || !aligned16(wt->wg) ||
+      !aligned16(wt->qk_norm_q) || !aligned16(wt->qk_norm_k) || !aligned16(wt->wo) ||
+      !aligned16(wt->norm_ffn) || !aligned16(wt->w13) || !aligned16(wt->w2) ||
+      (lin && !aligned16(lambda)) || !aligned16_or_null(state_out))
+    return SALA_ERR_INVALID_ARG;
+  if (ws_bytes < w.total || !aligned16(workspace)) return SALA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (w.d == 128) return run_block<128>(b, lin, sp, wt, lambda, x, y, state_out, ws, w, st);
+  return run_block<64>(b, lin, sp, wt, lambda, x, y, state_out, ws, w, st);
 }
 
 const char* sala_status_string(sala_status s) {

@@ -37,6 +37,7 @@ EXPORTED = [
     "sala_get_device_status", "sala_version", "sala_kernel_launch_count",
     "sala_sparse_select_noalloc", "sala_selftest_bounded_wait",
     "sala_sparse_select_begin", "sala_sparse_select_finish",
+    "sala_block_workspace_size", "sala_block_prefill",
 ]
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -65,6 +66,16 @@ class SparseDesc(ctypes.Structure):
 class DecodeDesc(ctypes.Structure):
     _fields_ = [("lin", LinearDesc), ("sp", SparseDesc), ("n_linear", ctypes.c_int),
                 ("cache_capacity", ctypes.c_int64)]
+
+
+class BlockDesc(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("ffn", ctypes.c_int), ("rms_eps", ctypes.c_float)]
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("norm_attn", "wq", "wk", "wv", "wg", "qk_norm_q", "qk_norm_k", "wo", "norm_ffn",
+                 "w13", "w2")]
 
 
 _PA = ctypes.c_void_p * SALA_MAX_LAYERS
@@ -100,6 +111,8 @@ def _load():
         "sala_selftest_bounded_wait": (I, [P]),
         "sala_sparse_select_begin": (I, [P] + [P] * 8 + [P]),
         "sala_sparse_select_finish": (I, [P, P, P, P, P]),
+        "sala_block_workspace_size": (S, [P, P, P]),
+        "sala_block_prefill": (I, [P, P, P, P, P, P, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -215,6 +228,31 @@ def sala_sparse_prefill(d: SparseDesc, q_norm, k_norm, v, gate, idx, out, worksp
     return LIB.sala_sparse_prefill(ctypes.byref(d), _ptr(q_norm), _ptr(k_norm), _ptr(v),
                                    _ptr(gate), _ptr(idx), _ptr(out), _ptr(workspace), ws_bytes,
                                    _stream(stream))
+
+
+def sala_block_workspace_size(b: BlockDesc, lin: Optional[LinearDesc] = None,
+                              sp: Optional[SparseDesc] = None) -> int:
+    return int(LIB.sala_block_workspace_size(ctypes.byref(b), None if lin is None else ctypes.byref(lin),
+                                             None if sp is None else ctypes.byref(sp)))
+
+
+def block_weights(w: dict) -> BlockWeights:
+    """ctypes view of a dict of device tensors (keys as BlockWeights' fields;
+    the tensors must stay alive while it is used)."""
+    bw = BlockWeights()
+    for name, _ in BlockWeights._fields_:
+        setattr(bw, name, _ptr(w[name]).value)
+    bw._keep = w
+    return bw
+
+
+def sala_block_prefill(b: BlockDesc, lin: Optional[LinearDesc], sp: Optional[SparseDesc],
+                       w: BlockWeights, lam, x, y, state_out, workspace, stream=None) -> int:
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return LIB.sala_block_prefill(ctypes.byref(b), None if lin is None else ctypes.byref(lin),
+                                  None if sp is None else ctypes.byref(sp), ctypes.byref(w),
+                                  _ptr(lam), _ptr(x), _ptr(y), _ptr(state_out), _ptr(workspace),
+                                  ws_bytes, _stream(stream))
 
 
 def sala_decode_workspace_size(d: DecodeDesc) -> int:

@@ -190,3 +190,23 @@ def decode_inputs(w: Workload, step: int, device="cpu"):
 def rms_weights(d: int, device="cpu"):
     """RMSNorm weights of every workload: all ones (no trained weights)."""
     return torch.ones(d, dtype=torch.float32, device=device)
+
+
+def block_weights(hidden: int, ffn: int, q_heads: int, kv_heads: int, head_dim: int, layer: int,
+                  device="cpu", seed: int = 0):
+    """Synthetic weights of one decoder block (no trained weights exist):
+    bf16 projections in the [out, in] layout drawn N(0, 1) / sqrt(in) from a
+    generator seeded with ``seed * 100 + 50 + layer`` (in the order wq, wk, wv,
+    wg, wo, w13, w2), all-ones norms.  The sub-block outputs are then of the
+    residual stream's order of magnitude."""
+    g = _gen(device, seed * 100 + 50 + layer)
+
+    def lin(out, inp):
+        return (torch.randn((out, inp), generator=g, device=device) / inp ** 0.5).to(torch.bfloat16)
+    w = {"wq": lin(q_heads * head_dim, hidden), "wk": lin(kv_heads * head_dim, hidden),
+         "wv": lin(kv_heads * head_dim, hidden), "wg": lin(q_heads * head_dim, hidden),
+         "wo": lin(hidden, q_heads * head_dim), "w13": lin(2 * ffn, hidden), "w2": lin(hidden, ffn)}
+    ones = lambda n: torch.ones(n, dtype=torch.float32, device=device)
+    w.update(norm_attn=ones(hidden), norm_ffn=ones(hidden), qk_norm_q=ones(head_dim),
+             qk_norm_k=ones(head_dim))
+    return w

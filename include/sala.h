@@ -198,6 +198,58 @@ sala_status sala_sparse_prefill(const sala_sparse_desc* d, const void* q_norm,
                                 const int32_t* idx, void* out, void* workspace,
                                 size_t ws_bytes, void* stream);
 
+/* -------------------------------------------------------------- full block */
+
+/* One SALA decoder block around one attention layer, over N tokens (no
+ * counterpart in the pages' numbers: it turns the attention-only throughput
+ * into a per-block figure of the kind of the pages' time to first token).
+ * The pages fix the structure in words (MiniCPM-SALA paper, section 2.1:
+ * every attention block is followed by an FFN block; summary: an output gate
+ * after each attention block); the rest is the plainest reading for the
+ * model family, with synthetic weights:
+ *   xn = RMSNorm(x) * norm_attn                     (fp32 math, bf16 out)
+ *   q, k, v, gate = xn Wq^T, xn Wk^T, xn Wv^T, xn Wg^T   (bf16, fp32 accum.)
+ *   a  = the linear (sala_linear_prefill) or sparse (sala_sparse_select +
+ *        sala_sparse_prefill) attention of q, k, v, gate
+ *   h  = x + a Wo^T                                  (fp32 residual stream)
+ *   hn = RMSNorm(h) * norm_ffn
+ *   y  = h + (silu(hn W1^T) * (hn W3^T)) W2^T
+ * The GEMMs run in cuBLASLt; norms, SwiGLU and the attention in this
+ * library's kernels. */
+typedef struct {
+  int hidden;        /* residual width = q_heads * head_dim of the attention  */
+  int ffn;           /* FFN inner width (a multiple of 8)                     */
+  float rms_eps;     /* of the two pre-norms                                  */
+} sala_block_desc;
+
+/* bf16 weights use the [out, in] row-major layout of a torch Linear. */
+typedef struct {
+  const float* norm_attn;   /* [hidden] fp32                                  */
+  const void* wq;           /* [Hq*d, hidden] bf16                            */
+  const void* wk;           /* [Hk*d, hidden] bf16 (Hk = heads for a linear   */
+  const void* wv;           /*   layer, kv_heads for the sparse one)          */
+  const void* wg;           /* [Hq*d, hidden] bf16                            */
+  const float* qk_norm_q;   /* [d] fp32 QK-RMSNorm weights of the attention   */
+  const float* qk_norm_k;   /* [d] fp32                                       */
+  const void* wo;           /* [hidden, Hq*d] bf16                            */
+  const float* norm_ffn;    /* [hidden] fp32                                  */
+  const void* w13;          /* [2*ffn, hidden] bf16: W1 rows, then W3 rows     */
+  const void* w2;           /* [hidden, ffn] bf16                             */
+} sala_block_weights;
+
+/* Exactly one of lin / sp is non-NULL and names the attention; its dtype
+ * must be SALA_BF16 and its seqlen / batch give the tokens. */
+size_t sala_block_workspace_size(const sala_block_desc* b, const sala_linear_desc* lin,
+                                 const sala_sparse_desc* sp);
+
+/* x, y: [B, N, hidden] fp32 (y must not alias x).  lambda: [H] fp32 for a
+ * linear layer (NULL for sparse).  state_out: optional [B, H, d, d] final
+ * linear state.  workspace: >= sala_block_workspace_size bytes. */
+sala_status sala_block_prefill(const sala_block_desc* b, const sala_linear_desc* lin,
+                               const sala_sparse_desc* sp, const sala_block_weights* w,
+                               const float* lambda, const float* x, float* y, float* state_out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------- decode */
 
 #define SALA_MAX_LAYERS 8

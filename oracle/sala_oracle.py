@@ -66,6 +66,7 @@ __all__ = [
     "sparse_attention_rows", "sparse_select_rows", "sparse_layer_rows",
     "token_softmax_importance", "select_token_softmax",
     "decode_linear_step", "decode_sparse_step",
+    "silu", "sala_block",
 ]
 
 F64 = np.float64
@@ -591,3 +592,53 @@ def decode_sparse_step(k_hist, v_hist, q, g, wq, wk, pos, *, block=64, topk=64, 
             p /= p.sum(axis=-1, keepdims=True)
             o[b, gg * G:(gg + 1) * G] = p @ V
     return sigmoid(g) * o, idx
+
+
+# ---------------------------------------------------------------------------
+# Full decoder block around the attention (synthetic weights)
+# ---------------------------------------------------------------------------
+
+def silu(x):
+    """x * sigmoid(x), the gate of the SwiGLU feed-forward network."""
+    x = np.asarray(x, F64)
+    return x / (1.0 + np.exp(-x))
+
+
+def sala_block(x, w, kind, *, q_heads, kv_heads, head_dim, eps=1e-6, lam=None, chunk=64,
+               pos0=0, rope_base=10000.0, block=64, topk=16, n_init=1, n_local=2):
+    """One SALA decoder block: attention sub-block and feed-forward sub-block,
+    each pre-normalised and added to the residual stream.
+
+    The pages fix the block structure only in words: every attention block
+    (linear or sparse) is followed by an FFN block (MiniCPM-SALA paper,
+    section 2.1), the attention output passes an output gate (summary).  The
+    rest is the plainest reading for a model of this family: RMSNorm before
+    each sub-block, bias-free projections q, k, v, gate from the normalised
+    input, the attention of this module (``linear_layer`` or
+    ``sparse_layer``), an output projection added to the residual, and a
+    SwiGLU FFN (silu(h W1^T) * (h W3^T)) W2^T added to the residual.
+
+    x: [B, N, hidden]; w: dict with norm_attn [hidden], wq [Hq*d, hidden],
+    wk / wv [Hkv*d, hidden], wg [Hq*d, hidden], qk_q / qk_k [d] (QK-RMSNorm
+    weights), wo [hidden, Hq*d], norm_ffn [hidden], w1 / w3 [ffn, hidden],
+    w2 [hidden, ffn] (torch Linear layout: [out, in]).  kind "linear" uses
+    q_heads for k and v too.  Returns y [B, N, hidden].
+    """
+    x = np.asarray(x, F64)
+    B, N, hidden = x.shape
+    W = {key: np.asarray(val, F64) for key, val in w.items()}
+    xn = rms_norm(x, W["norm_attn"], eps)
+    hk = q_heads if kind == "linear" else kv_heads
+    q = (xn @ W["wq"].T).reshape(B, N, q_heads, head_dim)
+    k = (xn @ W["wk"].T).reshape(B, N, hk, head_dim)
+    v = (xn @ W["wv"].T).reshape(B, N, hk, head_dim)
+    g = (xn @ W["wg"].T).reshape(B, N, q_heads, head_dim)
+    if kind == "linear":
+        a, _ = linear_layer(q, k, v, g, lam, W["qk_q"], W["qk_k"], chunk=chunk, pos0=pos0,
+                            rope_base=rope_base, eps=eps)
+    else:
+        a, _ = sparse_layer(q, k, v, g, W["qk_q"], W["qk_k"], block=block, topk=topk,
+                            n_init=n_init, n_local=n_local, eps=eps)
+    h = x + a.reshape(B, N, q_heads * head_dim) @ W["wo"].T
+    hn = rms_norm(h, W["norm_ffn"], eps)
+    return h + (silu(hn @ W["w1"].T) * (hn @ W["w3"].T)) @ W["w2"].T

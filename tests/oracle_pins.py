@@ -450,6 +450,48 @@ def check_decode_sparse(orc):
             assert [int(j) for j in idx[0, gg] if j >= 0] == want
 
 
+def check_silu(orc):
+    assert orc.silu(0.0) == 0.0
+    assert abs(float(orc.silu(2.0)) - 2.0 / (1.0 + math.exp(-2.0))) < 1e-15
+    assert abs(float(orc.silu(-40.0))) < 1e-15
+
+
+def check_sala_block_assembly(orc):
+    # The block against an independent scalar assembly on a tiny case: pre-
+    # norm, projections, the (already pinned) attention, output projection
+    # and residual, pre-norm, SwiGLU, residual.
+    r = _rng(19)
+    B, N, Hq, d, ff = 1, 8, 2, 4, 6
+    hid = Hq * d
+    x = r.standard_normal((B, N, hid))
+    w = {"norm_attn": 1 + 0.1 * r.standard_normal(hid), "wq": r.standard_normal((hid, hid)) / 3,
+         "wk": r.standard_normal((hid, hid)) / 3, "wv": r.standard_normal((hid, hid)) / 3,
+         "wg": r.standard_normal((hid, hid)) / 3, "qk_q": np.ones(d), "qk_k": np.ones(d),
+         "wo": r.standard_normal((hid, hid)) / 3, "norm_ffn": 1 + 0.1 * r.standard_normal(hid),
+         "w1": r.standard_normal((ff, hid)) / 3, "w3": r.standard_normal((ff, hid)) / 3,
+         "w2": r.standard_normal((hid, ff)) / 3}
+    lam = np.array([0.9, 1.0])
+    y = orc.sala_block(x, w, "linear", q_heads=Hq, kv_heads=Hq, head_dim=d, lam=lam, chunk=4)
+    def mv(m, v_):
+        return [sum(m[i][j] * v_[j] for j in range(len(v_))) for i in range(len(m))]
+    def nrm(v_, wt):
+        s_ = math.sqrt(sum(e * e for e in v_) / len(v_) + 1e-6)
+        return [e / s_ * wt[i] for i, e in enumerate(v_)]
+    xs = [list(x[0, t]) for t in range(N)]
+    proj = {k_: [mv(w[k_], nrm(xs[t], w["norm_attn"])) for t in range(N)]
+            for k_ in ("wq", "wk", "wv", "wg")}
+    rs = lambda key: np.array(proj[key]).reshape(1, N, Hq, d)
+    a, _ = orc.linear_layer(rs("wq"), rs("wk"), rs("wv"), rs("wg"), lam, np.ones(d), np.ones(d),
+                            chunk=4)
+    for t in range(N):
+        h = [xs[t][i] + e for i, e in enumerate(mv(w["wo"], list(a[0, t].reshape(-1))))]
+        hn = nrm(h, w["norm_ffn"])
+        u, g3 = mv(w["w1"], hn), mv(w["w3"], hn)
+        s_ = [u[i] / (1 + math.exp(-u[i])) * g3[i] for i in range(ff)]
+        want = [h[i] + e for i, e in enumerate(mv(w["w2"], s_))]
+        assert max(abs(y[0, t, i] - want[i]) for i in range(hid)) < 1e-10, t
+
+
 ALL_CHECKS = [
     check_rms_norm_closed_form, check_rms_norm_invariants, check_rope_complex,
     check_rope_invariants, check_sigmoid, check_linear_brute_force, check_linear_three_forms,
@@ -458,5 +500,5 @@ ALL_CHECKS = [
     check_sparse_select_exhaustive, check_sparse_rows_forms,
     check_token_softmax_selection, check_token_softmax_single_query,
     check_sparse_dense_limit, check_sparse_block_diagonal, check_sparse_masked_sdpa,
-    check_decode_linear, check_decode_sparse,
+    check_decode_linear, check_decode_sparse, check_silu, check_sala_block_assembly,
 ]

@@ -437,3 +437,39 @@ def test_split_selection_virtual_shards(sala):
     check_index_rows(gidx, ridx, scores, sp.topk, sp.n_init, sp.n_local)
     want = oracle.sigmoid(f64(g)) * oracle.sparse_attention(qh, kh, f64(v), gidx, 64)
     assert rel_err(f64(out), want) <= TOL
+
+
+@pytest.mark.parametrize("kind", ["linear", "sparse"])
+def test_block_prefill(sala, kind):
+    """One full decoder block (pre-norm, projections, the attention layer,
+    output projection and fp32 residual, pre-norm, SwiGLU FFN, residual)
+    through sala_block_prefill against the oracle's block.  The sparse
+    layer's top-k covers every candidate here, so its selection does not
+    depend on the bf16 rounding of the projected q and k (selection parity
+    is covered by the sparse-layer tests)."""
+    dev = torch.device("cuda")
+    N, Hq, d, ffn = 1024, 4, 128, 1024
+    hidden = Hq * d
+    Hk = Hq if kind == "linear" else 1
+    gen = torch.Generator(device=dev).manual_seed(21)
+    x = torch.randn((1, N, hidden), generator=gen, device=dev)
+    w = wl.block_weights(hidden, ffn, Hq, Hk, d, layer=0 if kind == "linear" else 3, device=dev)
+    bd = sala.BlockDesc(hidden, ffn, 1e-6)
+    lam = torch.tensor([0.9, 0.99, 1.0, 0.95], dtype=torch.float32, device=dev)
+    lin = sala.linear_desc(1, N, Hq, d, 64) if kind == "linear" else None
+    sp = None if kind == "linear" else sala.sparse_desc(1, N, Hq, Hk, d, topk=16, n_init=1,
+                                                        n_local=2)
+    ws = sala.workspace(sala.sala_block_workspace_size(bd, lin, sp), dev)
+    y = torch.empty_like(x)
+    st = sala.sala_block_prefill(bd, lin, sp, sala.block_weights(w), lam if lin else None, x, y,
+                                 None, ws)
+    assert st == sala.SALA_OK, sala.status_string(st)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    ref = oracle.sala_block(f64(x), {k_: f64(v_) for k_, v_ in w.items()}, kind, q_heads=Hq,
+                            kv_heads=Hk, head_dim=d, lam=f64(lam), chunk=64, block=64, topk=16,
+                            n_init=1, n_local=2)
+    # the block's own contribution (y - x), not dominated by the residual input
+    err = rel_err(f64(y) - f64(x), ref - f64(x))
+    print(f"block {kind}: rel err of y - x {err:.2e}")
+    assert err <= TOL, err

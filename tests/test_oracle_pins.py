@@ -60,6 +60,10 @@ MUTANTS = [
      "cand = np.arange(0, i + 1)\n                if len(cand) == 0:"),
     ("token importance without the softmax", "p = p / p.sum(axis=1, keepdims=True)\n                imp",
      "p = z\n                imp"),
+    ("block ffn gate and up swapped", "(silu(hn @ W[\"w1\"].T) * (hn @ W[\"w3\"].T))",
+     "(silu(hn @ W[\"w3\"].T) * (hn @ W[\"w1\"].T))"),
+    ("block residual dropped", "h = x + a.reshape(B, N, q_heads * head_dim) @ W[\"wo\"].T",
+     "h = a.reshape(B, N, q_heads * head_dim) @ W[\"wo\"].T"),
     ("decode query group sum", "qg = qh_s[b, gg * G:(gg + 1) * G].sum(axis=0, dtype=sd)",
      "qg = qh_s[b, gg * G]"),
 ]
