@@ -466,7 +466,11 @@ def test_block_prefill(sala, kind):
     assert st == sala.SALA_OK, sala.status_string(st)
     torch.cuda.synchronize()
     assert sala.sala_get_device_status() == 0
-    ref = oracle.sala_block(f64(x), {k_: f64(v_) for k_, v_ in w.items()}, kind, q_heads=Hq,
+    wf = {k_: f64(v_) for k_, v_ in w.items()}
+    wf.update(qk_q=wf.pop("qk_norm_q"), qk_k=wf.pop("qk_norm_k"))
+    w13 = wf.pop("w13")
+    wf.update(w1=w13[:ffn], w3=w13[ffn:])
+    ref = oracle.sala_block(f64(x), wf, kind, q_heads=Hq,
                             kv_heads=Hk, head_dim=d, lam=f64(lam), chunk=64, block=64, topk=16,
                             n_init=1, n_local=2)
     # the block's own contribution (y - x), not dominated by the residual input
