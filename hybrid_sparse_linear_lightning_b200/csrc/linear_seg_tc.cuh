@@ -233,9 +233,11 @@ struct LsSumLayout {
   static constexpr int kPw = kLsSumStages * kStage;  // lam^m, m = 0..128
   static constexpr int kBar = kPw + 4 * 132;         // ld_full[S], ld_empty[S], k_ready[S], done
   static constexpr int kMisc = kBar + 8 * (3 * kLsSumStages + 1);
-  static constexpr int kW = kMisc + 16;              // RMSNorm weights of k, 128 floats
+  // 16-byte aligned: both arrays are read with 16-byte vector loads
+  static constexpr int kW = (kMisc + 16 + 15) / 16 * 16;   // RMSNorm weights of k, 128 floats
   static constexpr int kTh = kW + 512;               // RoPE frequencies, 64 floats
   static constexpr int kBytes = kTh + 256;
+  static_assert(kW % 16 == 0 && kTh % 16 == 0 && kBar % 8 == 0, "shared-memory alignment");
 };
 
 __global__ void __launch_bounds__(kLsSumThreads, 1)
@@ -436,8 +438,10 @@ struct LsOutLayout {
   // s_smem_full, s_smem_empty, o_full[2], o_empty[2], fin, qk_ready
   static constexpr int kNumBars = 4 + 8 + 4 + 1 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
-  static constexpr int kW = kMisc + 16;                  // RMSNorm weights of q, k: 2 x 128 floats
+  // 16-byte aligned: read with 16-byte vector loads
+  static constexpr int kW = (kMisc + 16 + 15) / 16 * 16;  // RMSNorm weights of q, k: 2 x 128 floats
   static constexpr int kBytes = kW + 1024;
+  static_assert(kW % 16 == 0 && kBar % 8 == 0, "shared-memory alignment");
   // TMEM columns
   static constexpr int kColQK = 0;     // Q^ K^T; P (bf16 pairs) overwrites its first 64 columns
   static constexpr int kColO = 128;    // O of tile c in columns 128 + 128 (c & 1)
