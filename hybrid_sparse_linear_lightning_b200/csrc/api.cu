@@ -185,10 +185,12 @@ sala_status run_select_finish(const sala_sparse_desc* d, const float* qsum, cons
                               int32_t* idx, cudaStream_t st) {
   const int nb = d->seqlen / d->block;
   const int width = d->topk + d->n_init + d->n_local;
-  const size_t smem = (size_t)nb * sizeof(uint32_t);
+  const int tq = select_rows_per_cta(nb);
+  const size_t smem = (size_t)tq * nb * sizeof(uint32_t);
   if (allow_smem(select_topk_kernel<D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
-  select_topk_kernel<D><<<d->batch * d->kv_heads * nb, kSelectThreads, smem, st>>>(
-      qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width);
+  const int n_tiles = (nb + tq - 1) / tq;
+  select_topk_kernel<D><<<d->batch * d->kv_heads * n_tiles, kSelectThreads, smem, st>>>(
+      qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width, tq);
   return launch_status();
 }
 

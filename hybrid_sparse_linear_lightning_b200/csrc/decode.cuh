@@ -16,9 +16,8 @@
 // persistent grid of one CTA per SM whose phases are separated by bounded
 // grid barriers (the launch is cooperative, so every CTA is resident):
 //
-//   P0  every linear (layer, batch, head) state update and output; the
-//       sparse layer's cache append and query normalisation; the scores of
-//       all candidate blocks in chunks of 256, each score also counted in a
+//   P0  the sparse layer's cache append and query normalisation; the scores
+//       of all candidate blocks in chunks of 256, each score also counted in a
 //       4096-bin histogram of its top 12 key bits per (batch, kv head).  The
 //       CTA that scores the last chunk of a (batch, kv head) then selects
 //       for it while the other CTAs finish their units: the bin T holding
@@ -30,7 +29,9 @@
 //       select over all scores.
 //   B1  barrier.
 //   P1  one unit per (batch, kv head, selected block): partial softmax sums
-//       of the group's q heads over that block's keys.
+//       of the group's q heads over that block's keys; then every linear
+//       (layer, batch, head) state update and output, which need nothing
+//       from the sparse layer and fill the phase's tail.
 //   B2  barrier.
 //   P2  one unit per (batch, q head): combine of the partials, output gate.
 //
@@ -59,14 +60,37 @@ constexpr int kDecMaxLayers = 8;
 // number of scored chunks.
 constexpr int kDecCtlBarriers = 2;
 constexpr int kDecLine = 32;            // words per 128-byte line
-__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (2 * kDecCtlBarriers + 1 + bg); }
+__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (2 * kDecCtlBarriers + 2 + bg); }
 __device__ __forceinline__ unsigned* dec_bar_count(unsigned* ctl, int i) { return ctl + kDecLine * i; }
 __device__ __forceinline__ unsigned* dec_bar_flag(unsigned* ctl, int i) {
   return ctl + kDecLine * (kDecCtlBarriers + i);
 }
-__device__ __forceinline__ unsigned* dec_work(unsigned* ctl) { return ctl + kDecLine * 2 * kDecCtlBarriers; }
+// work counters of P0 (phase 0) and P1 (phase 1)
+__device__ __forceinline__ unsigned* dec_work(unsigned* ctl, int phase) {
+  return ctl + kDecLine * (2 * kDecCtlBarriers + phase);
+}
 __device__ __forceinline__ unsigned* dec_bg_done(unsigned* ctl, int bg) {
-  return ctl + kDecLine * (2 * kDecCtlBarriers + 1 + bg);
+  return ctl + kDecLine * (2 * kDecCtlBarriers + 2 + bg);
+}
+
+// Persistent loop over `n` units taken from a work counter in order; the CTA
+// asks for its next unit while it works on the current one.  f(u) runs with
+// the whole CTA.
+template <typename F>
+__device__ __forceinline__ void dec_unit_loop(unsigned* counter, int n, F f) {
+  __shared__ int s_unit;
+  if (threadIdx.x == 0) s_unit = (int)atomicAdd(counter, 1u);
+  __syncthreads();
+  int u = s_unit;
+  while (u < n) {
+    unsigned nxt = 0;
+    if (threadIdx.x == 0) nxt = atomicAdd(counter, 1u);
+    f(u);
+    __syncthreads();
+    if (threadIdx.x == 0) s_unit = (int)nxt;
+    __syncthreads();
+    u = s_unit;
+  }
 }
 
 struct DecodeParams {
@@ -722,33 +746,24 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
 
   // P0: scores + histogram (+ selection by the last chunk of each (b, g)),
   // linear layers, sparse prep; direct index rows when nothing ranks
-  // Units are handed out by a work counter in order (scores first, so that
-  // the selections start early), each CTA asking for its next unit while it
-  // works on the current one.
+  // P0, units from a work counter in order (scores first, so that the
+  // selections start early): scores + histograms (+ selection by the CTA that
+  // scores the last chunk of each (b, g)), the sparse layer's cache append and
+  // queries, direct index rows when nothing ranks.
   const int n_direct = ranked ? 0 : BG;
-  const int n_p0 = n_score + n_lin + p.B + n_direct;
-  __shared__ int s_unit;
-  if (threadIdx.x == 0) s_unit = (int)atomicAdd(dec_work(p.ctl), 1u);
-  __syncthreads();
-  int u = s_unit;
-  while (u < n_p0) {
-    unsigned nxt = 0;
-    if (threadIdx.x == 0) nxt = atomicAdd(dec_work(p.ctl), 1u);
+  dec_unit_loop(dec_work(p.ctl, 0), n_score + p.B + n_direct, [&](int u) {
     if (u < n_score) dec_score_unit<T, D>(p, u, sm);
-    else if (u < n_score + n_lin) dec_linear_unit<T, D>(p, u - n_score, sm);
-    else if (u < n_score + n_lin + p.B) dec_sparse_prep_unit<T, D>(p, u - n_score - n_lin);
-    else dec_direct_row(p, u - n_score - n_lin - p.B);
-    __syncthreads();
-    if (threadIdx.x == 0) s_unit = (int)nxt;
-    __syncthreads();
-    u = s_unit;
-  }
+    else if (u < n_score + p.B) dec_sparse_prep_unit<T, D>(p, u - n_score);
+    else dec_direct_row(p, u - n_score - p.B);
+  });
   if (!dec_grid_sync(dec_bar_count(p.ctl, 0), dec_bar_flag(p.ctl, 0), [] {})) return;
-  // P1: attention partials
-  for (int u = blockIdx.x; u < BG * p.width; u += gridDim.x) {
-    dec_attn_unit<D>(p, u, dec_smem);
-    __syncthreads();
-  }
+  // P1: attention partials first, then the linear layers' state updates and
+  // outputs (independent of the sparse layer; they fill the phase's tail)
+  const int n_att = BG * p.width;
+  dec_unit_loop(dec_work(p.ctl, 1), n_att + n_lin, [&](int u) {
+    if (u < n_att) dec_attn_unit<D>(p, u, dec_smem);
+    else dec_linear_unit<T, D>(p, u - n_att, sm);
+  });
   if (!dec_grid_sync(dec_bar_count(p.ctl, 1), dec_bar_flag(p.ctl, 1), [] {})) return;
   // P2: combine and gate
   for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {

@@ -129,55 +129,89 @@ __device__ __forceinline__ void topk_emit_sorted(const uint32_t* keys, int n_can
   }
 }
 
-// One CTA per (batch, kv head g, query block i).  Dynamic smem: n_b uint32 keys.
+// One CTA per (batch, kv head g, TQ consecutive query blocks i0..i0+TQ-1).
+// Each candidate block mean is read once per CTA and scored against the TQ
+// group queries (one warp per candidate; every score is the same lane-strided
+// fmaf chain and butterfly sum whatever TQ is, so the keys do not depend on
+// the tiling).  Then the rows' top-k are taken one after the other.
+// Dynamic smem: TQ * nb uint32 keys.
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads)
 select_topk_kernel(const float* __restrict__ qsum, const float* __restrict__ kbar,
                    int32_t* __restrict__ idx, int nb, int Hkv, int topk, int n_init,
-                   int n_local, int width) {
+                   int n_local, int width, int TQ) {
   extern __shared__ uint32_t keys[];
-  __shared__ float qv[D];
+  __shared__ float qv[8][D];
   __shared__ int hist[256];
   __shared__ int scan_scratch[kSelectThreads / 32 + 1];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
 
-  const int i = blockIdx.x % nb;
-  const int g = (blockIdx.x / nb) % Hkv;
-  const int b = blockIdx.x / (nb * Hkv);
+  const int n_tiles = (nb + TQ - 1) / TQ;
+  const int i0 = (blockIdx.x % n_tiles) * TQ;
+  const int g = (blockIdx.x / n_tiles) % Hkv;
+  const int b = blockIdx.x / (n_tiles * Hkv);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
+  const int nq = min(TQ, nb - i0);
 
-  const int n_cand = max(0, i - n_local + 1 - n_init);
-  const int k = min(topk, n_cand);
-  // initial blocks
-  const int n_first = min(n_init, i + 1);
-  for (int e = tid; e < n_first; e += kSelectThreads) row[e] = e;
-  const int local_lo = max(n_init, i - n_local + 1);
-  const int n_loc = max(0, i - local_lo + 1);
-  for (int e = tid; e < n_loc; e += kSelectThreads) row[n_first + k + e] = local_lo + e;
-  for (int e = n_first + k + n_loc + tid; e < width; e += kSelectThreads) row[e] = -1;
-  if (k == 0) return;
-  if (k == n_cand) {
-    for (int e = tid; e < n_cand; e += kSelectThreads) row[n_first + e] = n_init + e;
-    return;
+  // rows that rank (fewer slots than candidates) and the largest candidate count
+  int n_cand_max = 0;
+  for (int t = 0; t < nq; ++t) {
+    const int i = i0 + t;
+    int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
+    const int n_cand = max(0, i - n_local + 1 - n_init);
+    const int k = min(topk, n_cand);
+    const int n_first = min(n_init, i + 1);
+    const int local_lo = max(n_init, i - n_local + 1);
+    const int n_loc = max(0, i - local_lo + 1);
+    for (int e = tid; e < n_first; e += kSelectThreads) row[e] = e;
+    for (int e = tid; e < n_loc; e += kSelectThreads) row[n_first + k + e] = local_lo + e;
+    for (int e = n_first + k + n_loc + tid; e < width; e += kSelectThreads) row[e] = -1;
+    if (k == n_cand)
+      for (int e = tid; e < n_cand; e += kSelectThreads) row[n_first + e] = n_init + e;
+    if (k > 0 && k < n_cand) n_cand_max = n_cand;
   }
+  if (n_cand_max == 0) return;
 
-  // scores of the candidates, one warp per candidate row (coalesced over d)
-  for (int e = tid; e < D; e += kSelectThreads) qv[e] = qsum[(((long long)b * nb + i) * Hkv + g) * D + e];
+  // scores: one warp per candidate, TQ queries (coalesced over d)
+  for (int e = tid; e < nq * D; e += kSelectThreads) {
+    const int t = e / D, d = e % D;
+    qv[t][d] = qsum[(((long long)b * nb + i0 + t) * Hkv + g) * D + d];
+  }
   __syncthreads();
   const float inv_sqrt_d = rsqrtf((float)D);
-  for (int c = warp; c < n_cand; c += kSelectThreads / 32) {
+  for (int c = warp; c < n_cand_max; c += kSelectThreads / 32) {
     const float* kr = kbar + (((long long)b * nb + n_init + c) * Hkv + g) * D;
-    float p = 0.f;
+    float kk[D / 32];
 #pragma unroll
-    for (int e = lane; e < D; e += 32) p = fmaf(qv[e], kr[e], p);
-    p = warp_sum(p);
-    if (lane == 0) keys[c] = score_key(p * inv_sqrt_d);
+    for (int u = 0; u < D / 32; ++u) kk[u] = kr[lane + 32 * u];
+    for (int t = 0; t < nq; ++t) {
+      float p = 0.f;
+#pragma unroll
+      for (int u = 0; u < D / 32; ++u) p = fmaf(qv[t][lane + 32 * u], kk[u], p);
+      p = warp_sum(p);
+      if (lane == 0) keys[t * nb + c] = score_key(p * inv_sqrt_d);
+    }
   }
   __syncthreads();
 
-  topk_emit_sorted(keys, n_cand, k, row + n_first, n_init, hist, scan_scratch, &s_prefix, &s_need);
+  for (int t = 0; t < nq; ++t) {
+    const int i = i0 + t;
+    const int n_cand = max(0, i - n_local + 1 - n_init);
+    const int k = min(topk, n_cand);
+    if (k == 0 || k == n_cand) continue;           // uniform across the CTA
+    int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
+    const int n_first = min(n_init, i + 1);
+    topk_emit_sorted(keys + t * nb, n_cand, k, row + n_first, n_init, hist, scan_scratch,
+                     &s_prefix, &s_need);
+    __syncthreads();
+  }
+}
+
+// Query blocks per selection CTA: as many as fit 200 KB of keys, at most 8.
+inline int select_rows_per_cta(int nb) {
+  const int fit = (int)((200u << 10) / ((unsigned)nb * 4u));
+  return fit < 1 ? 1 : (fit > 8 ? 8 : fit);
 }
 
 }  // namespace sala
