@@ -175,7 +175,7 @@ __device__ __forceinline__ void sw128_norm_rope_half_row(uint8_t* tile, int r, i
   ss += __shfl_xor_sync(0xffffffffu, ss, 1);
   const float sc = rsqrtf(ss * (1.0f / 128) + eps) * f;
   const float rr = (float)r;
-#pragma unroll
+#pragma unroll 1
   for (int c4 = 0; c4 < 4; ++c4) {
     const int ch = 4 * h + c4;
     const int o = (ch ^ (r & 7)) << 4;
@@ -221,8 +221,8 @@ __device__ __forceinline__ void sw128_store_row32(uint8_t* tile, int r, int j, c
 // 1. Segment sums
 // --------------------------------------------------------------------------
 
-constexpr int kLsSumThreads = 640;     // warps 0-3: TMA, MMA, TMEM; 4-19: two scaling WGs of 8 warps
-constexpr int kLsSumScaleWGs = 2;
+constexpr int kLsSumThreads = 896;     // warps 0-3: TMA, MMA, TMEM; 4-27: three scaling WGs of 8 warps
+constexpr int kLsSumScaleWGs = 3;
 // One load stage per scaling warpgroup: stage a is only ever scaled by
 // warpgroup a, so each stage's barrier phases are consumed in order.
 constexpr int kLsSumStages = kLsSumScaleWGs;
