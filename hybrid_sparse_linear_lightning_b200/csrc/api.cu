@@ -179,19 +179,35 @@ sala_status run_select_begin(const sala_sparse_desc* d, const void* q, const voi
   return launch_status();
 }
 
+// SMs of the current device (cached per device).
+int device_sms() {
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  return sms[dev];
+}
+
 // Block-mean ranking of every query block from qsum and kbar.
 template <int D>
 sala_status run_select_finish(const sala_sparse_desc* d, const float* qsum, const float* kbar,
                               int32_t* idx, cudaStream_t st) {
   const int nb = d->seqlen / d->block;
   const int width = d->topk + d->n_init + d->n_local;
-  const int tq = select_rows_per_cta(nb);
-  const size_t smem = (size_t)tq * nb * sizeof(uint32_t);
-  if (allow_smem(select_topk_kernel<D>, smem) != cudaSuccess) return SALA_ERR_CUDA;
+  const int per = select_buffer_per(d->topk);
+  const int tq = select_rows_per_cta((long long)d->batch * d->kv_heads * nb, per, std::max(device_sms(), 1));
+  const size_t smem = (size_t)tq * per * kSelectThreads * 8;
   const int n_tiles = (nb + tq - 1) / tq;
-  select_topk_kernel<D><<<d->batch * d->kv_heads * n_tiles, kSelectThreads, smem, st>>>(
-      qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init, d->n_local, width, tq);
-  return launch_status();
+  const int grid = d->batch * d->kv_heads * n_tiles;
+  auto launch = [&](auto kern) {
+    if (allow_smem(kern, smem) != cudaSuccess) return SALA_ERR_CUDA;
+    kern<<<grid, kSelectThreads, smem, st>>>(qsum, kbar, idx, nb, d->kv_heads, d->topk, d->n_init,
+                                             d->n_local, width, tq);
+    return launch_status();
+  };
+  if (per == 2) return launch(select_topk_kernel<D, 2>);
+  if (per == 4) return launch(select_topk_kernel<D, 4>);
+  return launch(select_topk_kernel<D, 8>);
 }
 
 template <typename T, int D>
@@ -380,15 +396,6 @@ sala_status check_decode(const sala_decode_desc* d) {
   if (d->sp.q_heads > kDecodeMaxQHeads) return SALA_ERR_UNSUPPORTED;
   if (d->sp.selection != SALA_SELECT_BLOCK_MEAN) return SALA_ERR_UNSUPPORTED;
   return SALA_OK;
-}
-
-// SMs of the current device (cached per device).
-int device_sms() {
-  static int sms[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-  return sms[dev];
 }
 
 template <typename T, int D>

@@ -152,57 +152,6 @@ __device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const 
   }
 }
 
-// The same transform by two threads per row: lane pair (2k, 2k+1) of the
-// calling warp shares row r, the lane with h = lane & 1 takes chunk pairs
-// [4h, 4h + 4) (frequencies [32h, 32h + 32)); the mean square is combined
-// across the pair.  thsm: the 64 frequencies in shared memory.
-__device__ __forceinline__ void sw128_norm_rope_half_row(uint8_t* tile, int r, int h,
-                                                         const float* wsm, const float* thsm,
-                                                         float eps, float2 base, float f) {
-  uint8_t* row0 = tile + r * 128;
-  uint8_t* row1 = tile + 16384 + r * 128;
-  float ss = 0.f;
-#pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4) {
-    const int ch = 4 * h + c4;
-    const int o = (ch ^ (r & 7)) << 4;
-    float a[8], b[8];
-    load8(reinterpret_cast<const __nv_bfloat16*>(row0 + o), a);
-    load8(reinterpret_cast<const __nv_bfloat16*>(row1 + o), b);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
-  }
-  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-  const float sc = rsqrtf(ss * (1.0f / 128) + eps) * f;
-  const float rr = (float)r;
-#pragma unroll 1
-  for (int c4 = 0; c4 < 4; ++c4) {
-    const int ch = 4 * h + c4;
-    const int o = (ch ^ (r & 7)) << 4;
-    float a[8], b[8], wa[8], wb[8], th[8];
-    load8(reinterpret_cast<const __nv_bfloat16*>(row0 + o), a);
-    load8(reinterpret_cast<const __nv_bfloat16*>(row1 + o), b);
-    load8(wsm + ch * 8, wa);
-    load8(wsm + 64 + ch * 8, wb);
-    load8(thsm + ch * 8, th);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      // frequency i = 32 h + 8 c4 + e: its base angle sits in lane (i & 31) = 8 c4 + e
-      const float bx = __shfl_sync(0xffffffffu, base.x, 8 * c4 + e);
-      const float by = __shfl_sync(0xffffffffu, base.y, 8 * c4 + e);
-      const float x1 = a[e] * wa[e], x2 = b[e] * wb[e];
-      float sn, cs;
-      __sincosf(fmaf(rr, th[e], h ? by : bx), &sn, &cs);
-      cs *= sc;
-      sn *= sc;
-      a[e] = fmaf(x1, cs, -x2 * sn);
-      b[e] = fmaf(x2, cs, x1 * sn);
-    }
-    store8(reinterpret_cast<__nv_bfloat16*>(row0 + o), a);
-    store8(reinterpret_cast<__nv_bfloat16*>(row1 + o), b);
-  }
-}
-
 // 32 fp32 values -> bf16 columns [32 j, 32 j + 32) of row r of the same layout.
 __device__ __forceinline__ void sw128_store_row32(uint8_t* tile, int r, int j, const float* v) {
   uint8_t* atom = tile + (j >> 1) * 16384 + r * 128;
@@ -221,11 +170,8 @@ __device__ __forceinline__ void sw128_store_row32(uint8_t* tile, int r, int j, c
 // 1. Segment sums
 // --------------------------------------------------------------------------
 
-constexpr int kLsSumThreads = 896;     // warps 0-3: TMA, MMA, TMEM; 4-27: three scaling WGs of 8 warps
-constexpr int kLsSumScaleWGs = 3;
-// One load stage per scaling warpgroup: stage a is only ever scaled by
-// warpgroup a, so each stage's barrier phases are consumed in order.
-constexpr int kLsSumStages = kLsSumScaleWGs;
+constexpr int kLsSumThreads = 512;     // warps 0-3: TMA, MMA, TMEM; 4-15: one scaling WG per stage
+constexpr int kLsSumStages = 3;
 
 struct LsSumLayout {
   static constexpr int kStage = 65536;               // K^ tile, V tile (2 atoms x 16 KB each)
@@ -233,11 +179,10 @@ struct LsSumLayout {
   static constexpr int kPw = kLsSumStages * kStage;  // lam^m, m = 0..128
   static constexpr int kBar = kPw + 4 * 132;         // ld_full[S], ld_empty[S], k_ready[S], done
   static constexpr int kMisc = kBar + 8 * (3 * kLsSumStages + 1);
-  // 16-byte aligned: both arrays are read with 16-byte vector loads
+  // 16-byte aligned: read with 16-byte vector loads
   static constexpr int kW = (kMisc + 16 + 15) / 16 * 16;   // RMSNorm weights of k, 128 floats
-  static constexpr int kTh = kW + 512;               // RoPE frequencies, 64 floats
-  static constexpr int kBytes = kTh + 256;
-  static_assert(kW % 16 == 0 && kTh % 16 == 0 && kBar % 8 == 0, "shared-memory alignment");
+  static constexpr int kBytes = kW + 512;
+  static_assert(kW % 16 == 0 && kBar % 8 == 0, "shared-memory alignment");
 };
 
 __global__ void __launch_bounds__(kLsSumThreads, 1)
@@ -259,7 +204,6 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   float* pw = reinterpret_cast<float*>(smem + L::kPw);
   float* wsm = reinterpret_cast<float*>(smem + L::kW);
-  float* thsm = reinterpret_cast<float*>(smem + L::kTh);
 
   const int s = blockIdx.x % n_seg;
   const int h = (blockIdx.x / n_seg) % H;
@@ -275,14 +219,13 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
     for (int i = 0; i < kLsSumStages; ++i) {
       tc::mbar_init(ld_full + i, 1);
       tc::mbar_init(ld_empty + i, 1);
-      tc::mbar_init(k_ready + i, 8);
+      tc::mbar_init(k_ready + i, 4);
     }
     tc::mbar_init(done, 1);
     tc::fence_barrier_init();
   }
   if (threadIdx.x <= kLsTile) pw[threadIdx.x] = (float)pow((double)lam, (double)threadIdx.x);
   if (threadIdx.x < D) wsm[threadIdx.x] = wk[threadIdx.x];
-  if (threadIdx.x < 64) thsm[threadIdx.x] = rt.th[threadIdx.x];
   if (warp == 2) {
     tc::tmem_alloc(tmem_slot, 128);
     tc::tmem_relinquish();
@@ -328,16 +271,14 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
       tc::mma_commit(done);
     }
   } else if (warp >= 4) {
-    // scaling warpgroup a (8 warps, two threads per row) handles the tiles
-    // c = a, a + 2, ...; lane pair (2k, 2k+1) of local warp lw owns row
-    // 16 lw + k, each lane half of its chunk pairs
-    const int a = (warp - 4) >> 3;
-    const int lw = (warp - 4) & 7;
-    const int rrow = lw * 16 + (lane >> 1), half = lane & 1;
+    // scaling warpgroup a handles the tiles of stage a (c = a, a + 3, ...)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int a = (warp - 4) >> 2;
     const double2 th = rope_lane_freqs(rf);
     bool ok = true;
-    for (int c = a; ok && c < nt; c += kLsSumScaleWGs) {
-      const int st = a;                         // = c % kLsSumStages
+    for (int c = a; ok && c < nt; c += kLsSumStages) {
+      const int st = a;
       const int tile_start = (t0 + c) * kLsTile;
       const int Lt = min(kLsTile, N - tile_start);
       // k^_j (normalised, rotated at its position) scaled by
@@ -349,16 +290,14 @@ linear_segsum_kernel(const __grid_constant__ CUtensorMap kmap,
       const float2 base = rope_tile_base(pos0 + tile_start, th);
       ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + st, (c / kLsSumStages) & 1));
       if (!ok) break;
-      const float f = rrow < Lt ? ft * pw[Lt - 1 - rrow] : 0.f;
-      sw128_norm_rope_half_row(smem + st * L::kStage, rrow, half, wsm, thsm, eps, base, f);
+      const float f = r < Lt ? ft * pw[Lt - 1 - r] : 0.f;
+      sw128_norm_rope_row(smem + st * L::kStage, r, wsm, eps, base, rt, f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(k_ready + st);
     }
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    // dS (row r = key dim, 128 value columns) -> seg_state, by warps 4-7
-    if (warp < 8 && __all_sync(0xffffffffu, ok && tc::mbar_wait(done, 0))) {
+    // dS (row r = key dim, 128 value columns) -> seg_state, by warpgroup 0
+    if (a == 0 && __all_sync(0xffffffffu, ok && tc::mbar_wait(done, 0))) {
       tc::tc_fence_after();
       float* dst = seg_state + ((((long long)b * H + h) * n_seg + s) * D + r) * D;
       const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);

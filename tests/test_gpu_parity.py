@@ -197,6 +197,51 @@ def test_sparse_prefill_given_oracle_indices(sala):
     assert rel_err(f64(out), ref) <= TOL
 
 
+@pytest.mark.parametrize("topk", [16, 300, 700])
+@pytest.mark.parametrize("order", ["tied", "increasing", "decreasing"])
+def test_select_score_orders(sala, order, topk):
+    """Block scores that are all equal, that rise with the block index (every
+    candidate beats the ones before it) or that fall with it, over 1500
+    blocks, for top-k sizes of each selection buffer size.  Every key of
+    block j is the unit vector at angle theta_j in the plane of the first two
+    axes and every query is the first axis, so the score of block j is
+    proportional to cos(theta_j).  Equal scores keep the lowest blocks (the
+    tie rule, checked exactly); the other orders are checked against the
+    oracle's ranking within the tie window."""
+    dev = torch.device("cuda")
+    D, Hq, Hkv, nb, n_init, n_local = 128, 4, 2, 1500, 1, 2
+    N = nb * 64
+    if order == "tied":
+        th = torch.full((nb,), 0.7, dtype=torch.float64)
+    elif order == "increasing":
+        th = torch.linspace(1.4, 0.1, nb, dtype=torch.float64)
+    else:
+        th = torch.linspace(0.1, 1.4, nb, dtype=torch.float64)
+    kb = torch.zeros((nb, D), dtype=torch.float64)
+    kb[:, 0], kb[:, 1] = torch.cos(th), torch.sin(th)
+    k = kb.repeat_interleave(64, 0)[None, :, None, :].expand(1, N, Hkv, D)
+    k = k.to(dev, torch.bfloat16).contiguous()
+    q = torch.zeros((1, N, Hq, D), dtype=torch.bfloat16, device=dev)
+    q[..., 0] = 1.0
+    wt = torch.ones(D, dtype=torch.float32, device=dev)
+    _, _, _, idx = sala.sparse_select(q, k, wt, wt, topk=topk, n_init=n_init, n_local=n_local)
+    torch.cuda.synchronize()
+    assert sala.sala_get_device_status() == 0
+    gidx = idx.cpu().numpy()
+    _, _, _, ridx, scores = oracle.sparse_select(f64(q), f64(k), f64(wt), f64(wt), block=64,
+                                                 topk=topk, n_init=n_init, n_local=n_local)
+    check_index_rows(gidx, ridx, scores, topk, n_init, n_local)
+    if order == "tied":
+        for i in range(nb):
+            n_cand = max(0, i - n_local + 1 - n_init)
+            kk = min(topk, n_cand)
+            want = (list(range(min(n_init, i + 1))) + list(range(n_init, n_init + kk)) +
+                    list(range(max(n_init, i - n_local + 1), i + 1)))
+            want += [-1] * (gidx.shape[-1] - len(want))
+            for g in range(Hkv):
+                assert gidx[0, g, i].tolist() == want, (g, i)
+
+
 @pytest.mark.parametrize("case", ["one_block", "topk0", "local_covers_all", "mha", "init3"])
 def test_sparse_edges(sala, case):
     if case == "one_block":
