@@ -226,6 +226,7 @@ __device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* qh = sm;              // [kDecWarps][D] per-warp partial group sums
   float* qv = sm + kDecWarps * D;
+  unsigned* hs = reinterpret_cast<unsigned*>(qv + D);   // [kDecBins] this unit's histogram
   // this thread's half row of its candidate's block mean is loaded first, so
   // that the loads are in flight while the group query is formed
   const int c0 = ck * kDecChunk;
@@ -241,6 +242,7 @@ __device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
 #pragma unroll
     for (int e = 0; e < D / 8; ++e) kv[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  for (int e = tid; e < kDecBins; e += kDecThreads) hs[e] = 0u;
   float acc[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
@@ -275,7 +277,15 @@ __device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
   if (c < nc && half == 0) {
     const uint32_t key = score_key(s * rsqrtf((float)D));
     p.keys[(long long)bg * p.capb + c0 + c] = key;
-    atomicAdd(p.hist + (long long)bg * kDecBins + (key >> (32 - kDecBinBits)), 1u);
+    atomicAdd(hs + (key >> (32 - kDecBinBits)), 1u);
+  }
+  // the unit's histogram is added to the (b, g) one bin by bin, only where it
+  // is not empty: scores crowd into few bins, and a global atomic per score
+  // would queue on them
+  __syncthreads();
+  for (int e = tid; e < kDecBins; e += kDecThreads) {
+    const unsigned n = hs[e];
+    if (n) atomicAdd(p.hist + (long long)bg * kDecBins + e, n);
   }
   // the CTA that finishes the last chunk of (b, g) selects for it
   __shared__ int s_last_chunk;
@@ -774,7 +784,7 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
 
 // Dynamic shared memory of the step: the largest phase's need.
 inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int width) {
-  const size_t score = (size_t)(kDecWarps + 1) * D * 4;
+  const size_t score = (size_t)(kDecWarps + 1) * D * 4 + (size_t)kDecBins * 4;
   const size_t lin = (size_t)(3 * D + kDecThreads) * 4;
   const size_t attn = (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
                       (size_t)2 * G * D * 4 + (size_t)G * 8;
