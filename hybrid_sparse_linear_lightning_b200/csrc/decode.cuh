@@ -16,11 +16,14 @@
 // persistent grid of one CTA per SM whose phases are separated by bounded
 // grid barriers (the launch is cooperative, so every CTA is resident):
 //
-//   P0  the sparse layer's cache append and query normalisation; the scores
-//       of all candidate blocks in chunks of 256, each score also counted in a
-//       4096-bin histogram of its top 12 key bits per (batch, kv head).  The
-//       CTA that scores the last chunk of a (batch, kv head) then selects
-//       for it while the other CTAs finish their units: the bin T holding
+//   P0  the scores of all candidate blocks in chunks of 256, each score
+//       also counted in a 4096-bin histogram of its top 12 key bits per
+//       (batch, kv head); the sparse layer's cache append and query
+//       normalisation; then every linear (layer, batch, head) state update
+//       and output, which need nothing from the sparse layer and run while
+//       the selections do.  The CTA that scores the last chunk of a (batch,
+//       kv head) selects for it while the other CTAs take the remaining
+//       units: the bin T holding
 //       the k-th largest score, the candidates above T (certainly selected)
 //       and those in T (the boundary), the remaining ones picked exactly from
 //       the boundary (score descending, ties to the lower block), and the
@@ -29,9 +32,7 @@
 //       select over all scores.
 //   B1  barrier.
 //   P1  one unit per (batch, kv head, selected block): partial softmax sums
-//       of the group's q heads over that block's keys; then every linear
-//       (layer, batch, head) state update and output, which need nothing
-//       from the sparse layer and fill the phase's tail.
+//       of the group's q heads over that block's keys.
 //   B2  barrier.
 //   P2  one unit per (batch, q head): combine of the partials, output gate.
 //
@@ -73,21 +74,18 @@ __device__ __forceinline__ unsigned* dec_bg_done(unsigned* ctl, int bg) {
   return ctl + kDecLine * (2 * kDecCtlBarriers + 2 + bg);
 }
 
-// Persistent loop over `n` units taken from a work counter in order; the CTA
-// asks for its next unit while it works on the current one.  f(u) runs with
-// the whole CTA.
+// Persistent loop over `n` units in order: CTA x takes unit x first, and
+// later units from a work counter once it is free.  (Asking for the next
+// unit while the current one runs would let one CTA hold two units of the
+// first round while another has none.)  f(u) runs with the whole CTA.
 template <typename F>
 __device__ __forceinline__ void dec_unit_loop(unsigned* counter, int n, F f) {
   __shared__ int s_unit;
-  if (threadIdx.x == 0) s_unit = (int)atomicAdd(counter, 1u);
-  __syncthreads();
-  int u = s_unit;
+  int u = blockIdx.x;
   while (u < n) {
-    unsigned nxt = 0;
-    if (threadIdx.x == 0) nxt = atomicAdd(counter, 1u);
     f(u);
     __syncthreads();
-    if (threadIdx.x == 0) s_unit = (int)nxt;
+    if (threadIdx.x == 0) s_unit = (int)gridDim.x + (int)atomicAdd(counter, 1u);
     __syncthreads();
     u = s_unit;
   }
@@ -754,26 +752,21 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
   const int n_score = ranked ? BG * p.n_chunks : 0;
   const int n_lin = p.n_linear * p.B * p.H;
 
-  // P0: scores + histogram (+ selection by the last chunk of each (b, g)),
-  // linear layers, sparse prep; direct index rows when nothing ranks
-  // P0, units from a work counter in order (scores first, so that the
-  // selections start early): scores + histograms (+ selection by the CTA that
-  // scores the last chunk of each (b, g)), the sparse layer's cache append and
-  // queries, direct index rows when nothing ranks.
+  // P0, units in order (scores first, so that the selections start early):
+  // scores + histograms (+ selection by the CTA that scores the last chunk
+  // of each (b, g)), the sparse layer's cache append and queries, direct
+  // index rows when nothing ranks, the linear layers.
   const int n_direct = ranked ? 0 : BG;
-  dec_unit_loop(dec_work(p.ctl, 0), n_score + p.B + n_direct, [&](int u) {
+  dec_unit_loop(dec_work(p.ctl, 0), n_score + p.B + n_direct + n_lin, [&](int u) {
     if (u < n_score) dec_score_unit<T, D>(p, u, sm);
     else if (u < n_score + p.B) dec_sparse_prep_unit<T, D>(p, u - n_score);
-    else dec_direct_row(p, u - n_score - p.B);
+    else if (u < n_score + p.B + n_direct) dec_direct_row(p, u - n_score - p.B);
+    else dec_linear_unit<T, D>(p, u - n_score - p.B - n_direct, sm);
   });
   if (!dec_grid_sync(dec_bar_count(p.ctl, 0), dec_bar_flag(p.ctl, 0), [] {})) return;
-  // P1: attention partials first, then the linear layers' state updates and
-  // outputs (independent of the sparse layer; they fill the phase's tail)
+  // P1: attention partials
   const int n_att = BG * p.width;
-  dec_unit_loop(dec_work(p.ctl, 1), n_att + n_lin, [&](int u) {
-    if (u < n_att) dec_attn_unit<D>(p, u, dec_smem);
-    else dec_linear_unit<T, D>(p, u - n_att, sm);
-  });
+  dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit<D>(p, u, dec_smem); });
   if (!dec_grid_sync(dec_bar_count(p.ctl, 1), dec_bar_flag(p.ctl, 1), [] {})) return;
   // P2: combine and gate
   for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {
