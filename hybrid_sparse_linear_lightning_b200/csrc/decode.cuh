@@ -669,6 +669,163 @@ __device__ void dec_attn_unit(const DecodeParams& p, int u, unsigned char* smem_
   }
 }
 
+// The same partial sums on the tensor cores with warp-level MMAs
+// (m16n8k16, bf16 operands, fp32 accumulation), for groups of at most 16 q
+// heads: the group's queries (rows past G zero) against the block's 64 keys,
+// logits Q K^T by warps 0..7 (8 keys each), the softmax per head, then
+// P V by warps 0..D/8-1 (8 value columns each).  A 16-row tile is below the
+// smallest tcgen05 tile and the step is bound by latency, not by MMA
+// throughput.  Queries and P are rounded to bf16 for the products, as in the
+// prefill kernel.
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D>
+__device__ void dec_attn_unit_mma(const DecodeParams& p, int u, unsigned char* smem_raw) {
+  constexpr int NC = D / 8;
+  constexpr int DP = D + 4;
+  constexpr int QS = D + 8;            // bf16 row stride of Q (conflict-free fragment loads)
+  constexpr int PS = 64 + 8;           // bf16 row stride of P
+  const int slot = u % p.width;
+  const int bg = u / p.width;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  const int G = p.Hq / p.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint4* ks = reinterpret_cast<uint4*>(smem_raw);                 // [64][NC]
+  uint4* vs = ks + 64 * NC;                                       // [64][NC]
+  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(vs + 64 * NC);   // [16][QS]
+  float* lg = reinterpret_cast<float*>(qb + 16 * QS);             // [16][64]
+  __nv_bfloat16* pbs = reinterpret_cast<__nv_bfloat16*>(lg + 16 * 64);  // [16][PS]
+  float* pb = p.part + ((long long)bg * p.width + slot) * G * DP;
+  int j = __ldcg(p.idx + (long long)bg * p.width + slot);
+  if (j >= 0 && (long long)j * p.BLK > p.pos) {
+    set_status(kStatusBounds);
+    j = -1;
+  }
+  if (j < 0) {
+    for (int e = tid; e < G * DP; e += kDecThreads) pb[e] = (e % DP) == 0 ? -INFINITY : 0.f;
+    return;
+  }
+  const long long kend = min((long long)(j + 1) * p.BLK, p.pos + 1);
+  const int nk = (int)(kend - (long long)j * p.BLK);
+  {
+    // every load of the unit is issued before the first shared-memory store
+    constexpr int PER = (64 * NC + kDecThreads - 1) / kDecThreads;
+    uint4 kv[PER], vv[PER];
+#pragma unroll
+    for (int w = 0; w < PER; ++w) {
+      const int e = tid + w * kDecThreads, sr = e / NC, c = e % NC;
+      kv[w] = vv[w] = make_uint4(0, 0, 0, 0);
+      if (e < 64 * NC && sr < nk) {
+        const long long off = (((long long)b * p.cap + (long long)j * p.BLK + sr) * p.Hkv + g) * D + 8 * c;
+        kv[w] = __ldcg(reinterpret_cast<const uint4*>(p.k_cache + off));
+        vv[w] = __ldcg(reinterpret_cast<const uint4*>(p.v_cache + off));
+      }
+    }
+    // one query float4 per thread (16 x D / 4 <= 512)
+    const int qh = tid / (D / 4), qc = tid % (D / 4);
+    float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < 16 * D / 4 && qh < G)
+      qv = __ldcg(reinterpret_cast<const float4*>(p.qhat + ((long long)b * p.Hq + g * G + qh) * D) + qc);
+#pragma unroll
+    for (int w = 0; w < PER; ++w) {
+      const int e = tid + w * kDecThreads, sr = e / NC, c = e % NC;
+      if (e < 64 * NC) {
+        ks[sr * NC + (c ^ (sr & (NC - 1)))] = kv[w];
+        vs[sr * NC + (c ^ (sr & (NC - 1)))] = vv[w];
+      }
+    }
+    if (tid < 16 * D / 4) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(qv.x, qv.y), hi = __floats2bfloat162_rn(qv.z, qv.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(qb + qh * QS + 4 * qc) = pk;
+    }
+  }
+  __syncthreads();
+  const int fr = lane >> 2, fc = (lane & 3) * 2;     // fragment row / column pair
+  // logits: warp w < 8 takes keys [8w, 8w + 8)
+  if (warp < 8) {
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    const int sr = 8 * warp + fr;                      // this lane's key row (B operand)
+    const uint8_t* krow = reinterpret_cast<const uint8_t*>(ks + sr * NC);
+#pragma unroll
+    for (int kq = 0; kq < D / 16; ++kq) {
+      uint32_t a[4];
+      a[0] = *reinterpret_cast<const uint32_t*>(qb + fr * QS + 16 * kq + fc);
+      a[1] = *reinterpret_cast<const uint32_t*>(qb + (fr + 8) * QS + 16 * kq + fc);
+      a[2] = *reinterpret_cast<const uint32_t*>(qb + fr * QS + 16 * kq + 8 + fc);
+      a[3] = *reinterpret_cast<const uint32_t*>(qb + (fr + 8) * QS + 16 * kq + 8 + fc);
+      const uint32_t b0 = *reinterpret_cast<const uint32_t*>(
+          krow + (((2 * kq) ^ (sr & (NC - 1))) << 4) + 2 * fc);
+      const uint32_t b1 = *reinterpret_cast<const uint32_t*>(
+          krow + (((2 * kq + 1) ^ (sr & (NC - 1))) << 4) + 2 * fc);
+      mma_bf16_16816(c, a, b0, b1);
+    }
+    const int key = 8 * warp + fc;
+    lg[fr * 64 + key] = key < nk ? c[0] * p.sl2 : -INFINITY;
+    lg[fr * 64 + key + 1] = key + 1 < nk ? c[1] * p.sl2 : -INFINITY;
+    lg[(fr + 8) * 64 + key] = key < nk ? c[2] * p.sl2 : -INFINITY;
+    lg[(fr + 8) * 64 + key + 1] = key + 1 < nk ? c[3] * p.sl2 : -INFINITY;
+  }
+  __syncthreads();
+  // softmax of the block per head (one warp per row of the tile; rows past
+  // G get P = 0)
+  if (warp < 16) {
+    const int h = warp;
+    float p0 = 0.f, p1 = 0.f;
+    if (h < G) {
+      const float x0 = lg[h * 64 + lane], x1 = lg[h * 64 + lane + 32];
+      const float m = warp_max(fmaxf(x0, x1));      // key 0 is always valid: m is finite
+      p0 = exp2f(x0 - m);
+      p1 = exp2f(x1 - m);
+      const float l = warp_sum(p0 + p1);
+      if (lane < 4) pb[h * DP + lane] = lane == 0 ? m : (lane == 1 ? l : 0.f);
+    }
+    pbs[h * PS + lane] = __float2bfloat16_rn(p0);
+    pbs[h * PS + lane + 32] = __float2bfloat16_rn(p1);
+  }
+  __syncthreads();
+  // P V: warp w < D / 8 takes value columns [8w, 8w + 8)
+  if (warp < D / 8) {
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t vbase = (uint32_t)__cvta_generic_to_shared(vs);
+#pragma unroll
+    for (int kq = 0; kq < 4; ++kq) {
+      uint32_t a[4];
+      a[0] = *reinterpret_cast<const uint32_t*>(pbs + fr * PS + 16 * kq + fc);
+      a[1] = *reinterpret_cast<const uint32_t*>(pbs + (fr + 8) * PS + 16 * kq + fc);
+      a[2] = *reinterpret_cast<const uint32_t*>(pbs + fr * PS + 16 * kq + 8 + fc);
+      a[3] = *reinterpret_cast<const uint32_t*>(pbs + (fr + 8) * PS + 16 * kq + 8 + fc);
+      // rows (keys) 16 kq + 0..15 of value chunk `warp`, transposed into the
+      // B fragment: lanes 0-7 address keys 16kq+0..7, lanes 8-15 keys 16kq+8..15
+      const int key = 16 * kq + (lane & 15);
+      const uint32_t addr = vbase + (uint32_t)((key * NC + (warp ^ (key & (NC - 1)))) * 16);
+      uint32_t b0, b1;
+      asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
+                   : "=r"(b0), "=r"(b1)
+                   : "r"(addr));
+      mma_bf16_16816(c, a, b0, b1);
+    }
+    const int col = 8 * warp + fc;
+    if (fr < G) {
+      pb[fr * DP + 4 + col] = c[0];
+      pb[fr * DP + 4 + col + 1] = c[1];
+    }
+    if (fr + 8 < G) {
+      pb[(fr + 8) * DP + 4 + col] = c[2];
+      pb[(fr + 8) * DP + 4 + col + 1] = c[3];
+    }
+  }
+}
+
 // Combine of the `width` partials of q head hq of batch b and the output
 // gate.  Thread (quarter of the partials, column).
 template <typename T, int D>
@@ -766,7 +923,10 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
   if (!dec_grid_sync(dec_bar_count(p.ctl, 0), dec_bar_flag(p.ctl, 0), [] {})) return;
   // P1: attention partials
   const int n_att = BG * p.width;
-  dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit<D>(p, u, dec_smem); });
+  if (p.Hq / p.Hkv <= 16)
+    dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit_mma<D>(p, u, dec_smem); });
+  else
+    dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit<D>(p, u, dec_smem); });
   if (!dec_grid_sync(dec_bar_count(p.ctl, 1), dec_bar_flag(p.ctl, 1), [] {})) return;
   // P2: combine and gate
   for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {
@@ -779,8 +939,11 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
 inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int width) {
   const size_t score = (size_t)(kDecWarps + 1) * D * 4 + (size_t)kDecBins * 4;
   const size_t lin = (size_t)(3 * D + kDecThreads) * 4;
-  const size_t attn = (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
-                      (size_t)2 * G * D * 4 + (size_t)G * 8;
+  const size_t attn = G <= 16
+      ? (size_t)2 * 64 * D * 2 + (size_t)16 * (D + 8) * 2 + (size_t)16 * 64 * 4 +
+            (size_t)16 * (64 + 8) * 2                                     // dec_attn_unit_mma
+      : (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
+            (size_t)2 * G * D * 4 + (size_t)G * 8;                        // dec_attn_unit
   const size_t resolve = (size_t)2 * topk * 4 + 16 +
                          std::max((size_t)kDecBndMax * 8, (size_t)capb * 4);   // dec_select_bg
   const size_t comb = (size_t)2 * width * 4 + (size_t)(kDecThreads / D) * D * 4;
