@@ -371,7 +371,7 @@ DecodeWs decode_ws(const sala_decode_desc* d) {
   w.hist = w.ctl + align_up(dec_ctl_words((int)BG) * 4);
   w.keys = w.hist + align_up(BG * kDecBins * 4);
   w.zero_bytes = w.keys;                         // control words and histograms
-  w.idx = w.keys + align_up(BG * capb * 4);
+  w.idx = w.keys + align_up(BG * dec_key_stride((long long)capb) * 4);
   w.qhat = w.idx + align_up(BG * width * 4);
   w.part = w.qhat + align_up(B * Hq * D * 4);
   w.total = w.part + align_up(BG * width * G * (D + 4) * 4);
@@ -428,6 +428,7 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   p.n_local = S.n_local; p.width = S.topk + S.n_init + S.n_local;
   p.cap = d->cache_capacity;
   p.capb = d->cache_capacity / S.block;
+  p.kstride = dec_key_stride(p.capb);
   p.pos = cur_len;
   p.eps_s = S.rms_eps;
   p.sl2 = sparse_scale(&S) * 1.4426950408889634f;
@@ -445,7 +446,7 @@ sala_status run_decode(const sala_decode_desc* d, const sala_decode_io* io, void
   // barrier counters, per-(batch, kv head) counts and histograms start at zero
   if (cudaMemsetAsync(ws, 0, w.zero_bytes, st) != cudaSuccess) return SALA_ERR_CUDA;
   const int G = S.q_heads / S.kv_heads;
-  const size_t smem = decode_smem_bytes(D, G, S.topk, p.capb, p.width);
+  const size_t smem = decode_smem_bytes(D, G, S.topk, p.kstride, p.width);
   auto kern = decode_step_kernel<T, D>;
   if (allow_smem(kern, smem) != cudaSuccess) return SALA_ERR_CUDA;
   int per_sm = 0;

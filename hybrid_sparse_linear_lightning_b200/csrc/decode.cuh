@@ -55,6 +55,11 @@ constexpr int kDecBndMax = 1024;        // boundary entries resolved by rank cou
 constexpr int kDecodeMaxQHeads = 64;    // largest sparse-layer q head count the step takes
 constexpr int kDecMaxLayers = 8;
 
+// Row stride (in keys) of the per-(batch, kv head) score keys: rows start on
+// 16-byte boundaries so that the selection can stage a row with 16-byte
+// asynchronous copies.
+__host__ __device__ constexpr long long dec_key_stride(long long capb) { return (capb + 3) / 4 * 4; }
+
 // Control words at the start of the workspace (zeroed by the host before
 // each launch), each on its own 128-byte line: the barriers' arrival counts
 // and release flags, the P0 work counter, and per (batch, kv head) the
@@ -118,13 +123,14 @@ struct DecodeParams {
   float* ksum;
   int Hq, Hkv, BLK, topk, n_init, n_local, width;
   long long cap, capb, pos;
+  long long kstride;    // row stride of `keys`: capb rounded up to 16 bytes
   float eps_s, sl2;
   // selection shape of this step (the same for every batch and kv head)
   int bcur, n_cand, kk, n_chunks;
   // workspace
   unsigned* ctl;
   unsigned* hist;       // [B * Hkv][kDecBins]
-  uint32_t* keys;       // [B * Hkv][capb]
+  uint32_t* keys;       // [B * Hkv][kstride]
   int* idx;             // [B * Hkv][width]
   float* qhat;          // [B][Hq][D]
   float* part;          // [B * Hkv][width][G][D + 4]
@@ -274,7 +280,7 @@ __device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
   s += __shfl_xor_sync(0xffffffffu, s, 1);
   if (c < nc && half == 0) {
     const uint32_t key = score_key(s * rsqrtf((float)D));
-    p.keys[(long long)bg * p.capb + c0 + c] = key;
+    p.keys[(long long)bg * p.kstride + c0 + c] = key;
     atomicAdd(hs + (key >> (32 - kDecBinBits)), 1u);
   }
   // the unit's histogram is added to the (b, g) one bin by bin, only where it
@@ -452,6 +458,18 @@ __device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem
   uint8_t* tail = reinterpret_cast<uint8_t*>(sorted + p.topk);
   tail = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tail) + 15) & ~uintptr_t(15));
   uint2* sb = reinterpret_cast<uint2*>(tail);                     // [kDecBndMax] boundary
+  uint32_t* sk = reinterpret_cast<uint32_t*>(tail + kDecBndMax * 8);  // [kstride] all keys
+  // 0. every key of (b, g) is copied into shared memory while the threshold
+  // is found (L2 -> shared, 16 bytes a copy, rows 16-byte aligned)
+  {
+    const uint32_t* src = p.keys + (long long)bg * p.kstride;
+    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(sk);
+    for (int e = tid; e < (p.n_cand + 3) / 4; e += kDecThreads)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst + 16 * e),
+                   "l"(src + 4 * e)
+                   : "memory");
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  }
   // 1. threshold bin
   {
     const unsigned* h = p.hist + (long long)bg * kDecBins;
@@ -473,27 +491,18 @@ __device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem
   }
   // 2. above / boundary lists (slot order is arbitrary; the result is not)
   const unsigned T = (unsigned)s_T;
-  constexpr int kBatch = 16;            // keys in flight per thread
-  for (int c0 = 0; c0 < p.n_cand; c0 += kBatch * kDecThreads) {
-    uint32_t kv[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int c = c0 + u * kDecThreads + tid;
-      kv[u] = c < p.n_cand ? __ldcg(p.keys + (long long)bg * p.capb + c) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int c = c0 + u * kDecThreads + tid;
-      if (c >= p.n_cand) continue;
-      const unsigned bin = kv[u] >> (32 - kDecBinBits);
-      if (bin > T) {
-        const int slot = atomicAdd(&s_n_above, 1);
-        if (slot < p.topk) chosen[slot] = c;
-        else set_status(kStatusBounds);
-      } else if (bin == T) {
-        const int slot = atomicAdd(&s_n_bnd, 1);
-        if (slot < kDecBndMax) sb[slot] = make_uint2(kv[u], (unsigned)c);
-      }
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  __syncthreads();
+  for (int c = tid; c < p.n_cand; c += kDecThreads) {
+    const uint32_t key = sk[c];
+    const unsigned bin = key >> (32 - kDecBinBits);
+    if (bin > T) {
+      const int slot = atomicAdd(&s_n_above, 1);
+      if (slot < p.topk) chosen[slot] = c;
+      else set_status(kStatusBounds);
+    } else if (bin == T) {
+      const int slot = atomicAdd(&s_n_bnd, 1);
+      if (slot < kDecBndMax) sb[slot] = make_uint2(key, (unsigned)c);
     }
   }
   __syncthreads();
@@ -514,10 +523,6 @@ __device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem
     }
   } else {
     // degenerate boundary: exact radix select over every key of (b, g)
-    uint32_t* sk = reinterpret_cast<uint32_t*>(tail);
-    __syncthreads();
-    for (int e = tid; e < p.n_cand; e += kDecThreads) sk[e] = __ldcg(p.keys + (long long)bg * p.capb + e);
-    __syncthreads();
     topk_emit_sorted<kDecThreads>(sk, p.n_cand, p.kk, sorted, 0, hist_s, scan_s, &s_prefix,
                                   &s_need);
     in_order = true;
@@ -852,6 +857,8 @@ __device__ void dec_combine_unit(const DecodeParams& p, int u, float* sm) {
     const int e = qtr + v * NQ;
     pv[v] = e < p.width ? __ldcg(pb + e * pstride + 4 + col) : 0.f;
   }
+  const long long off = ((long long)b * p.Hq + hq) * D + tid;
+  const float gt = tid < D ? ldf<T>(p.gate, off) : 0.f;     // the gate, loaded up front
   for (int e = tid; e < p.width; e += kDecThreads) {
     wts[e] = __ldcg(pb + e * pstride);
     lsum[e] = __ldcg(pb + e * pstride + 1);
@@ -891,9 +898,8 @@ __device__ void dec_combine_unit(const DecodeParams& p, int u, float* sm) {
     float acc = 0.f;
 #pragma unroll
     for (int r = 0; r < NQ; ++r) acc += red[r * D + tid];
-    const long long off = ((long long)b * p.Hq + hq) * D + tid;
     const float inv = s_l > 0.f ? 1.f / s_l : 0.f;
-    static_cast<T*>(p.out)[off] = from_f32<T>(sigmoidf_(ldf<T>(p.gate, off)) * acc * inv);
+    static_cast<T*>(p.out)[off] = from_f32<T>(sigmoidf_(gt) * acc * inv);
   }
 }
 
@@ -936,7 +942,7 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
 }
 
 // Dynamic shared memory of the step: the largest phase's need.
-inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int width) {
+inline size_t decode_smem_bytes(int D, int G, int topk, long long kstride, int width) {
   const size_t score = (size_t)(kDecWarps + 1) * D * 4 + (size_t)kDecBins * 4;
   const size_t lin = (size_t)(3 * D + kDecThreads) * 4;
   const size_t attn = G <= 16
@@ -945,7 +951,7 @@ inline size_t decode_smem_bytes(int D, int G, int topk, long long capb, int widt
       : (size_t)2 * 64 * D * 2 + (size_t)G * D * 4 + (size_t)G * 64 * 4 +
             (size_t)2 * G * D * 4 + (size_t)G * 8;                        // dec_attn_unit
   const size_t resolve = (size_t)2 * topk * 4 + 16 +
-                         std::max((size_t)kDecBndMax * 8, (size_t)capb * 4);   // dec_select_bg
+                         (size_t)kDecBndMax * 8 + (size_t)kstride * 4;   // dec_select_bg
   const size_t comb = (size_t)2 * width * 4 + (size_t)(kDecThreads / D) * D * 4;
   return std::max(std::max(std::max(score, lin), std::max(attn, resolve)), comb);
 }
