@@ -475,7 +475,15 @@ __device__ void dec_select_bg(const DecodeParams& p, int bg, unsigned char* smem
     const unsigned* h = p.hist + (long long)bg * kDecBins;
     int cnt[8], tot = 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) { cnt[u] = (int)__ldcg(h + kDecBins - 1 - 8 * tid - u); tot += cnt[u]; }
+    for (int u = 0; u < 8; ++u) cnt[u] = 0;
+    {
+      // this thread's 8 bins kDecBins-1-8 tid .. kDecBins-8-8 tid as two 16-byte loads
+      const uint4* hv = reinterpret_cast<const uint4*>(h + kDecBins - 8 - 8 * tid);
+      const uint4 lo = __ldcg(hv), hi = __ldcg(hv + 1);
+      const unsigned w[8] = {hi.w, hi.z, hi.y, hi.x, lo.w, lo.z, lo.y, lo.x};
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { cnt[u] = (int)w[u]; tot += cnt[u]; }
+    }
     if (tid == 0) { s_n_above = 0; s_n_bnd = 0; s_T = 0; }
     int all;
     const int before = block_exclusive_scan<kDecThreads>(tot, scan_s, &all);
