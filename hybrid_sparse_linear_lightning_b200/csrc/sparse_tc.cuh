@@ -96,6 +96,34 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- setup: barriers, TMEM, the block list
+  if (warp == 0) {
+    // valid prefix of the ascending index row (entries in [0, i]), read by
+    // the whole warp 32 entries at a time: it ends at the first -1 or at the
+    // first entry out of range or out of order (which also sets the bounds bit)
+    const int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
+    int n = 0, prev = -1;
+    for (int e0 = 0; e0 < width; e0 += 32) {
+      const int e = e0 + lane;
+      const int j = e < width ? __ldg(row + e) : -1;
+      int jp = __shfl_up_sync(0xffffffffu, j, 1);
+      if (lane == 0) jp = prev;
+      const bool good = j >= 0 && j <= i && j > jp;
+      const unsigned gm = __ballot_sync(0xffffffffu, good);
+      const int run = gm == 0xffffffffu ? 32 : __ffs(~gm) - 1;   // leading good lanes
+      if (lane < run) sel[n + lane] = j;
+      const int jstop = __shfl_sync(0xffffffffu, j, run & 31);
+      if (run < 32 && jstop >= 0 && lane == 0) set_status(kStatusBounds);
+      n += run;
+      prev = __shfl_sync(0xffffffffu, j, (run + 31) & 31);
+      if (run < 32) break;
+    }
+    // a valid row lists at least the query's own block; an empty row gets a
+    // zero output and the bounds bit
+    if (lane == 0) {
+      if (n == 0) set_status(kStatusBounds);
+      *n_sel_slot = n;
+    }
+  }
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
     for (int s = 0; s < kSpTcStages; ++s) {
@@ -111,20 +139,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     }
     tc::mbar_init(fin, 1);
     tc::fence_barrier_init();
-    // valid prefix of the ascending index row (entries in [0, i])
-    const int32_t* row = idx + (((long long)b * Hkv + g) * nb + i) * width;
-    int n = 0, prev = -1;
-    for (int e = 0; e < width; ++e) {
-      const int j = row[e];
-      if (j < 0) break;
-      if (j > i || j <= prev) { set_status(kStatusBounds); break; }
-      sel[n++] = j;
-      prev = j;
-    }
-    // a valid row lists at least the query's own block; an empty row gets a
-    // zero output and the bounds bit
-    if (n == 0) set_status(kStatusBounds);
-    *n_sel_slot = n;
   }
   if (warp == 2) {
     tc::tmem_alloc(tmem_slot, L::kTmemCols);
