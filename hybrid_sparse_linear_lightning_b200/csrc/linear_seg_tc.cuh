@@ -390,13 +390,13 @@ struct LsOutLayout {
 // Warpgroup roles: warpgroup 0 holds the TMA producer (warp 0), the MMA
 // issuer (warp 1, one elected thread) and the TMEM owner (warp 2) and gives
 // registers away (56 per thread); warpgroups 1-3 take them (152 per thread):
-// warpgroup 1 normalises and rotates the raw Q rows of each tile in place,
-// then rescales Q^ into Q' and builds P (one warp per TMEM lane quadrant),
-// warpgroup 2 normalises and rotates the raw K rows, rescales K^ into K' and
-// carries the state (fp32 in TMEM; a bf16 copy in shared memory is the B
-// operand of the next Q' S product),
-// warpgroup 3 runs the gated epilogue of tile c while tile c + 1 accumulates
-// into the other O buffer.  56 x 128 + 152 x 384 = 65536 = 128 x 512, the
+// warpgroup 1 normalises and rotates the raw Q rows of each tile in place and
+// rescales Q^ into Q', warpgroup 2 does the same for K; warpgroup 3 (one warp
+// per TMEM lane quadrant) builds P, carries the state (fp32 in TMEM; a bf16
+// copy in shared memory is the B operand of the next Q' S product) and runs
+// the gated epilogue of tile c while tile c + 1 accumulates into the other O
+// buffer.  The row transforms of tile c + 1 thus run while P, P V and the
+// epilogue of tile c do.  56 x 128 + 152 x 384 = 65536 = 128 x 512, the
 // registers the block is launched with (the host checks the 128).
 constexpr int kLsOutRegsLaunch = 128;
 constexpr int kLsOutRegsLow = 56;
@@ -564,32 +564,87 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       }
     }
 
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ P (warps 4-7)
+  } else if (warp < 12) {
+    // -------------------------------------------- Q (warps 4-7) / K (warps 8-11)
+    // Normalise and rotate the raw rows of each tile in place, then rescale
+    // them into Q' / K' once Q^ K^T has read the tile.  Nothing else: the
+    // transform of tile c + 1 runs while warps 12-15 build P of tile c.
     tc::setmaxnreg_inc<kLsOutRegsHigh>();
-    // Row quadrant q has 32-column chunks 0..q on or below the diagonal; chunk
-    // u of P (bf16 pairs) lands on columns [16 u, 16 u + 16) of the same rows,
-    // which were read with chunk u / 2 <= u, so each chunk is written back as
-    // soon as it is built.
+    const bool is_k = warp >= 8;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const int part = is_k ? L::kK : L::kQ;
+    const float* w = wsm + (is_k ? D : 0);
     const double2 th = rope_lane_freqs(rf);
     for (int c = 0; c < nt; ++c) {
-      // raw q row -> q^ (RMSNorm, RoPE at its position), in place
+      const int Lt = tile_len(c);
+      // raw row -> q^ / k^ (RMSNorm, RoPE at its position), in place
       const float2 base = rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, th);
       if (!__all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1))) break;
-      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kQ, r, wsm, eps, base, rt, 1.f);
+      sw128_norm_rope_row(smem + (c & 1) * L::kStage + part, r, w, eps, base, rt, 1.f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qk_ready);
       if (!__all_sync(0xffffffffu, tc::mbar_wait(qk_full, c & 1))) break;
-      // Q'_r = lam^(r+1) q^_r once Q^ K^T has read the tile
-      sw128_scale_row(smem + (c & 1) * L::kStage + L::kQ, r, pw[r + 1]);
+      // Q'_r = lam^(r+1) q^_r;  K'_r = lam^(L-1-r) k^_r (0 past the end)
+      const float f = is_k ? (r < Lt ? pw[Lt - 1 - r] : 0.f) : pw[r + 1];
+      sw128_scale_row(smem + (c & 1) * L::kStage + part, r, f);
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qk_scaled);
-      // P_rj = QK_rj lam^(r-j) for j <= r (rows past the end are never stored)
+    }
+  } else {
+    // ------------------------------------- P, state and gated epilogue (warps 12-15)
+    tc::setmaxnreg_inc<kLsOutRegsHigh>();
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;     // token row of P and O; key-dim row of S
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    // S_start: bf16 copy for the first Q^ S product, lam^L0 S_start into TMEM
+    {
+      const float* src = seg_state + ((((long long)b * H + h) * n_seg + s) * D + r) * D;
+      const float f0 = pw[tile_len(0)];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float x[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 t = *reinterpret_cast<const float4*>(src + 32 * j + e);
+          x[e] = t.x; x[e + 1] = t.y; x[e + 2] = t.z; x[e + 3] = t.w;
+        }
+        sw128_store_row32(smem + L::kS, r, j, x);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] *= f0;
+        tc::tmem_st32(lane_base + L::kColS + 32 * j, x);
+      }
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(s_smem_full);
+        tc::mbar_arrive(s_scaled);
+      }
+    }
+    constexpr int kGW = 16 * (int)sizeof(T) / 16;     // 16-byte words per 16 gate values
+    // The gate tile of tile c + 1 is pulled into L2 by a bulk tensor prefetch
+    // while tile c is written out; each thread then loads its whole gate row
+    // before waiting for the accumulator.
+    auto prefetch_gate = [&](int c) {
+      if (warp == 12 && lane == 0 && c < nt) {
+        const int row = b * N + (t0 + c) * kLsTile;
+        tc::tma_prefetch_l2_2d(&gmap, h * D, row);
+        tc::tma_prefetch_l2_2d(&gmap, h * D + 64, row);
+      }
+    };
+    if (warp == 12 && lane == 0) tc::tma_prefetch(&gmap);
+    prefetch_gate(0);
+    for (int c = 0; c < nt; ++c) {
+      // ---- P_rj = QK_rj lam^(r-j) for j <= r (rows past the end are never stored)
+      // Row quadrant q has 32-column chunks 0..q on or below the diagonal; chunk
+      // u of P (bf16 pairs) lands on columns [16 u, 16 u + 16) of the same rows,
+      // which were read with chunk u / 2 <= u, so each chunk is written back as
+      // soon as it is built.
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(qk_full, c & 1))) break;
       tc::tc_fence_after();
 #pragma unroll
       for (int q0 = 0; q0 < 4; ++q0) {
@@ -624,104 +679,33 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(p_full);
-    }
-  } else if (warp < 12) {
-    // ------------------------------------------------------------ K' and state
-    tc::setmaxnreg_inc<kLsOutRegsHigh>();
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;     // token row of K'; key-dim row of S
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    // S_start: bf16 copy for the first Q^ S product, lam^L0 S_start into TMEM
-    {
-      const float* src = seg_state + ((((long long)b * H + h) * n_seg + s) * D + r) * D;
-      const float f0 = pw[tile_len(0)];
+      // ---- S_c: bf16 copy for the next Q^ S product, lam^L(c+1) S_c back into TMEM
+      if (c + 1 < nt) {
+        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(s_full, c & 1));
+        if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(s_smem_empty, c & 1));
+        if (!ok) break;
+        tc::tc_fence_after();
+        const float f = pw[tile_len(c + 1)];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float x[32];
+        for (int j = 0; j < 4; ++j) {
+          float x[32];
+          tc::tmem_ld32(lane_base + L::kColS + 32 * j, x);
+          tc::tmem_wait_ld();
+          sw128_store_row32(smem + L::kS, r, j, x);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 t = *reinterpret_cast<const float4*>(src + 32 * j + e);
-          x[e] = t.x; x[e + 1] = t.y; x[e + 2] = t.z; x[e + 3] = t.w;
+          for (int e = 0; e < 32; ++e) x[e] *= f;
+          tc::tmem_st32(lane_base + L::kColS + 32 * j, x);
         }
-        sw128_store_row32(smem + L::kS, r, j, x);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] *= f0;
-        tc::tmem_st32(lane_base + L::kColS + 32 * j, x);
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc::mbar_arrive(s_smem_full);
+          tc::mbar_arrive(s_scaled);
+        }
       }
-      tc::tmem_wait_st();
-      tc::tc_fence_before();
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tc::mbar_arrive(s_smem_full);
-        tc::mbar_arrive(s_scaled);
-      }
-    }
-    bool ok = true;
-    const double2 th = rope_lane_freqs(rf);
-    for (int c = 0; ok && c < nt; ++c) {
-      const int Lt = tile_len(c);
-      // raw k row -> k^ (RMSNorm, RoPE at its position), in place
-      const float2 base = rope_tile_base(pos0 + (long long)(t0 + c) * kLsTile, th);
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(ld_full + (c & 1), (c >> 1) & 1));
-      if (!ok) break;
-      sw128_norm_rope_row(smem + (c & 1) * L::kStage + L::kK, r, wsm + D, eps, base, rt, 1.f);
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(qk_ready);
-      // K'_r = lam^(L-1-r) k^_r (0 past the end) once Q^ K^T has read the tile
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(qk_full, c & 1));
-      if (!ok) break;
-      sw128_scale_row(smem + (c & 1) * L::kStage + L::kK, r, r < Lt ? pw[Lt - 1 - r] : 0.f);
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(qk_scaled);
-      if (c + 1 == nt) break;
-      // S_c: bf16 copy for the next Q^ S product, lam^L(c+1) S_c back into TMEM
-      ok = __all_sync(0xffffffffu, tc::mbar_wait(s_full, c & 1));
-      if (ok) ok = __all_sync(0xffffffffu, tc::mbar_wait(s_smem_empty, c & 1));
-      if (!ok) break;
-      tc::tc_fence_after();
-      const float f = pw[tile_len(c + 1)];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float x[32];
-        tc::tmem_ld32(lane_base + L::kColS + 32 * j, x);
-        tc::tmem_wait_ld();
-        sw128_store_row32(smem + L::kS, r, j, x);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] *= f;
-        tc::tmem_st32(lane_base + L::kColS + 32 * j, x);
-      }
-      tc::tmem_wait_st();
-      tc::tc_fence_before();
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tc::mbar_arrive(s_smem_full);
-        tc::mbar_arrive(s_scaled);
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ gated epilogue
-    tc::setmaxnreg_inc<kLsOutRegsHigh>();
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;     // token row of O
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    constexpr int kGW = 16 * (int)sizeof(T) / 16;     // 16-byte words per 16 gate values
-    // The gate tile of tile c + 1 is pulled into L2 by a bulk tensor prefetch
-    // while tile c is written out; each thread then loads its whole gate row
-    // before waiting for the accumulator.
-    auto prefetch_gate = [&](int c) {
-      if (warp == 12 && lane == 0 && c < nt) {
-        const int row = b * N + (t0 + c) * kLsTile;
-        tc::tma_prefetch_l2_2d(&gmap, h * D, row);
-        tc::tma_prefetch_l2_2d(&gmap, h * D + 64, row);
-      }
-    };
-    if (warp == 12 && lane == 0) tc::tma_prefetch(&gmap);
-    prefetch_gate(0);
-    for (int c = 0; c < nt; ++c) {
+      // ---- gated epilogue of tile c
       prefetch_gate(c + 1);
       const bool valid = r < tile_len(c);
       const long long row_off = (((long long)b * N + (long long)(t0 + c) * kLsTile + r) * H + h) * D;
