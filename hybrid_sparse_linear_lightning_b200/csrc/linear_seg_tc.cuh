@@ -34,6 +34,8 @@
 // runs out sets the device status word and the CTA winds down.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "prologue.cuh"
 #include "tc_ptx.cuh"
@@ -626,6 +628,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
       }
     }
     constexpr int kGW = 16 * (int)sizeof(T) / 16;     // 16-byte words per 16 gate values
+    const float2 hs2 = make_float2(0.5f * scale, 0.5f * scale);
     // The gate tile of tile c + 1 is pulled into L2 by a bulk tensor prefetch
     // while tile c is written out; each thread then loads its whole gate row
     // before waiting for the accumulator.
@@ -732,14 +735,35 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
           if (lane == 0) tc::mbar_arrive(o_empty + (c & 1));
         }
         if (valid) {
-          const T* g = reinterpret_cast<const T*>(graw[j]);
+          if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+            // out = (s/2 + s/2 tanh(g/2)) o = s sigmoid(g) o, in f32x2 pairs
 #pragma unroll
-          for (int e = 0; e < 16; e += 8) {
-            float gv[8], o8[8];
-            load8(g + e, gv);
+            for (int e = 0; e < 2; ++e) {
+              const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&graw[j][e]);
+              uint4 res;
+              __nv_bfloat162* r2 = reinterpret_cast<__nv_bfloat162*>(&res);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) o8[u] = sigmoid_tanh(gv[u]) * (scale * ov[e + u]);
-            store8(dst + 16 * j + e, o8);
+              for (int u = 0; u < 4; ++u) {
+                const float2 hg = __fmul2_rn(__bfloat1622float2(g2[u]), make_float2(0.5f, 0.5f));
+                float tx, ty;
+                asm("tanh.approx.f32 %0, %1;" : "=f"(tx) : "f"(hg.x));
+                asm("tanh.approx.f32 %0, %1;" : "=f"(ty) : "f"(hg.y));
+                const float2 sg = __ffma2_rn(make_float2(tx, ty), hs2, hs2);
+                const float2 ou = __fmul2_rn(sg, make_float2(ov[8 * e + 2 * u], ov[8 * e + 2 * u + 1]));
+                r2[u] = __floats2bfloat162_rn(ou.x, ou.y);
+              }
+              *reinterpret_cast<uint4*>(dst + 16 * j + 8 * e) = res;
+            }
+          } else {
+            const T* g = reinterpret_cast<const T*>(graw[j]);
+#pragma unroll
+            for (int e = 0; e < 16; e += 8) {
+              float gv[8], o8[8];
+              load8(g + e, gv);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) o8[u] = sigmoid_tanh(gv[u]) * (scale * ov[e + u]);
+              store8(dst + 16 * j + e, o8);
+            }
           }
         }
       }
