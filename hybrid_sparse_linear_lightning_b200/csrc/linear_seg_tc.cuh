@@ -660,11 +660,16 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
 #pragma unroll
             for (int e = 0; e < 32; ++e) xv[e] = e <= lane ? xv[e] * pw[lane - e] : 0.f;
           } else {
-            float dcy = pw[r - 32 * q0 - 31];
+            // element e decays by lam^(r - 32 q0 - e): pairs (e, e + 1) from the top
+            const int a = r - 32 * q0;
+            float2 dcy = make_float2(pw[a - 30], pw[a - 31]);
+            const float2 l2 = make_float2(pw[2], pw[2]);
 #pragma unroll
-            for (int e = 31; e >= 0; --e) {
-              xv[e] *= dcy;
-              dcy *= lam;
+            for (int e = 30; e >= 0; e -= 2) {
+              const float2 y = __fmul2_rn(make_float2(xv[e], xv[e + 1]), dcy);
+              xv[e] = y.x;
+              xv[e + 1] = y.y;
+              dcy = __fmul2_rn(dcy, l2);
             }
           }
 #pragma unroll
@@ -689,6 +694,7 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
         if (!ok) break;
         tc::tc_fence_after();
         const float f = pw[tile_len(c + 1)];
+        const float2 f2 = make_float2(f, f);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float x[32];
@@ -696,7 +702,11 @@ linear_segout_kernel(const __grid_constant__ CUtensorMap qmap,
           tc::tmem_wait_ld();
           sw128_store_row32(smem + L::kS, r, j, x);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] *= f;
+          for (int e = 0; e < 32; e += 2) {
+            const float2 y = __fmul2_rn(make_float2(x[e], x[e + 1]), f2);
+            x[e] = y.x;
+            x[e + 1] = y.y;
+          }
           tc::tmem_st32(lane_base + L::kColS + 32 * j, x);
         }
         tc::tmem_wait_st();
