@@ -140,14 +140,17 @@ __device__ __forceinline__ void sw128_norm_rope_row(uint8_t* tile, int r, const 
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i = ch * 8 + e;
-      const float x1 = a[e] * wa[e], x2 = b[e] * wb[e];
+      // (x1, x2) = the pair (i, i + 64) times its weights; (c, s) = sc (cos, sin)
+      const float2 x = __fmul2_rn(make_float2(a[e], b[e]), make_float2(wa[e], wb[e]));
       const float b0 = __shfl_sync(0xffffffffu, i < 32 ? base.x : base.y, i & 31);
       float sn, cs;
       __sincosf(fmaf(rr, rt.th[i], b0), &sn, &cs);
-      cs *= sc;
-      sn *= sc;
-      a[e] = fmaf(x1, cs, -x2 * sn);
-      b[e] = fmaf(x2, cs, x1 * sn);
+      const float2 cr = __fmul2_rn(make_float2(cs, sn), make_float2(sc, sc));
+      // (x1 c - x2 s, x2 c + x1 s)
+      const float2 y = __ffma2_rn(make_float2(x.x, x.y), make_float2(cr.x, cr.x),
+                                  __fmul2_rn(make_float2(x.y, x.x), make_float2(-cr.y, cr.y)));
+      a[e] = y.x;
+      b[e] = y.y;
     }
     store8(reinterpret_cast<__nv_bfloat16*>(row0 + o), a);
     store8(reinterpret_cast<__nv_bfloat16*>(row1 + o), b);
