@@ -95,7 +95,36 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   const int hbase = g * G + hq * kSpTcHeadsPerCta;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- setup: barriers, TMEM, the block list
+  // ---- setup: barriers, the Q tiles (loaded at once: they do not depend on
+  // the block list), TMEM, the block list
+  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sKV = smem + L::kKVBase;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int s = 0; s < kSpTcStages; ++s) {
+      tc::mbar_init(kv_full + s, 1);
+      tc::mbar_init(kv_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      tc::mbar_init(s_full + 2 * t, 1);
+      tc::mbar_init(s_full + 2 * t + 1, 1);
+      tc::mbar_init(p_full + t, 4);
+      tc::mbar_init(o_done + 2 * t, 1);
+      tc::mbar_init(o_done + 2 * t + 1, 1);
+    }
+    tc::mbar_init(fin, 1);
+    tc::fence_barrier_init();
+    tc::tma_prefetch(&qmap);
+    tc::tma_prefetch(&kmap);
+    tc::tma_prefetch(&vmap);
+    tc::mbar_expect_tx(q_full, 2 * L::kQTile);
+    const int row0 = b * N + i * 64;
+    for (int t = 0; t < 2; ++t)
+      for (int hl = 0; hl < 2; ++hl)
+        for (int a = 0; a < L::kAtoms; ++a)
+          tc::tma_load_2d(sQ + t * L::kQTile + a * (128 * 128) + hl * (64 * 128), &qmap, q_full,
+                          (hbase + 2 * t + hl) * D + 64 * a, row0);
+  }
   if (warp == 0) {
     // valid prefix of the ascending index row (entries in [0, i]), read by
     // the whole warp 32 entries at a time: it ends at the first -1 or at the
@@ -124,22 +153,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       *n_sel_slot = n;
     }
   }
-  if (threadIdx.x == 0) {
-    tc::mbar_init(q_full, 1);
-    for (int s = 0; s < kSpTcStages; ++s) {
-      tc::mbar_init(kv_full + s, 1);
-      tc::mbar_init(kv_empty + s, 1);
-    }
-    for (int t = 0; t < 2; ++t) {
-      tc::mbar_init(s_full + 2 * t, 1);
-      tc::mbar_init(s_full + 2 * t + 1, 1);
-      tc::mbar_init(p_full + t, 4);
-      tc::mbar_init(o_done + 2 * t, 1);
-      tc::mbar_init(o_done + 2 * t + 1, 1);
-    }
-    tc::mbar_init(fin, 1);
-    tc::fence_barrier_init();
-  }
   if (warp == 2) {
     tc::tmem_alloc(tmem_slot, L::kTmemCols);
     tc::tmem_relinquish();
@@ -150,22 +163,13 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   const uint32_t tmem = *tmem_slot;
   const int n_sel = *n_sel_slot;
 
-  uint8_t* sQ = smem + L::kQ;
-  uint8_t* sKV = smem + L::kKVBase;
-
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    if (tc::elect_one() && n_sel == 0) {
+      // nothing reads the Q tiles: let their load land before the CTA ends
+      tc::mbar_wait(q_full, 0);
+    }
     if (tc::elect_one() && n_sel > 0) {
-      tc::tma_prefetch(&qmap);
-      tc::tma_prefetch(&kmap);
-      tc::tma_prefetch(&vmap);
-      tc::mbar_expect_tx(q_full, 2 * L::kQTile);
-      const int row0 = b * N + i * 64;
-      for (int t = 0; t < 2; ++t)
-        for (int hl = 0; hl < 2; ++hl)
-          for (int a = 0; a < L::kAtoms; ++a)
-            tc::tma_load_2d(sQ + t * L::kQTile + a * (128 * 128) + hl * (64 * 128), &qmap, q_full,
-                            (hbase + 2 * t + hl) * D + 64 * a, row0);
       for (int j = 0; j < n_sel; ++j) {
         const int st = j % kSpTcStages, use = j / kSpTcStages;
         if (use > 0 && !tc::mbar_wait(kv_empty + st, (use - 1) & 1)) break;
