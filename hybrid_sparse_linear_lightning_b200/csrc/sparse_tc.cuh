@@ -76,9 +76,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* s_full = kv_empty + kSpTcStages;   // [tile * 2 + buffer]
   uint64_t* p_full = s_full + 4;
   // P V of block j of tile t completes o_done[2 t + (j & 1)]: every wait on it
-  // (for block j-1, by the MMA issuer before S of block j+1, by the softmax
-  // before a rescale and before the epilogue) comes after P V of block j-3
-  // has completed, so a parity wait is never more than one phase behind
+  // (for block j-1, by the softmax before a rescale and before the epilogue)
+  // comes after P V of block j-3 has completed, so a parity wait is never
+  // more than one phase behind
   uint64_t* o_done = p_full + 2;
   uint64_t* fin = o_done + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -223,13 +223,12 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       for (int j = 0; ok && j < n_sel; ++j) {
         if (j + 1 < n_sel) {
           if (!(ok = tc::mbar_wait(kv_full + (j + 1) % kSpTcStages, ((j + 1) / kSpTcStages) & 1))) break;
-          for (int t = 0; t < 2 && ok; ++t) {
-            // buffer (j+1) & 1 last held P of block j-1
-            if (j >= 1 && !(ok = tc::mbar_wait(o_done + 2 * t + ((j - 1) & 1), ((j - 1) >> 1) & 1))) break;
-            tc::tc_fence_after();
-            issue_s(t, j + 1);
-          }
-          if (!ok) break;
+          // buffer (j+1) & 1 last held P of block j-1, read by P V of block
+          // j-1; that MMA was issued before this one by this thread, and
+          // tcgen05.mma operations from one thread execute in issue order, so
+          // S of block j+1 needs no wait for it
+          tc::tc_fence_after();
+          for (int t = 0; t < 2; ++t) issue_s(t, j + 1);
         }
         for (int t = 0; t < 2 && ok; ++t) {
           if (!(ok = tc::mbar_wait(p_full + t, j & 1))) break;
