@@ -45,9 +45,9 @@ struct SpTcLayout {
   static constexpr int kQ = 0;
   static constexpr int kKVBase = kQ + 2 * kQTile;
   static constexpr int kBar = kKVBase + kSpTcStages * 2 * kKV;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_full[2],
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[tile][buf], p_full[tile][buf],
   // o_done[tile][block parity], fin
-  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 4 + 2 + 4 + 1;
+  static constexpr int kNumBars = 1 + 2 * kSpTcStages + 4 + 4 + 4 + 1;
   static constexpr int kMisc = kBar + 8 * kNumBars;
   static constexpr int kSel = kMisc + 16;               // int sel[width]
   static constexpr int kBytes(int width) { return kSel + 4 * width; }
@@ -74,12 +74,19 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kSpTcStages;
   uint64_t* s_full = kv_empty + kSpTcStages;   // [tile * 2 + buffer]
+  // P of block j of tile t is published on p_full[2 t + (j & 1)]. The softmax
+  // of a tile can finish blocks j and j+1 while the MMA issuer still waits for
+  // the other tile's block j (S of block j+1 is issued before that wait), but
+  // not block j+2 (its S is issued after it): with one barrier per buffer
+  // parity each barrier is at most one phase ahead of its waiter, where a
+  // single barrier per tile could be two phases ahead and its parity wait
+  // would never return
   uint64_t* p_full = s_full + 4;
   // P V of block j of tile t completes o_done[2 t + (j & 1)]: every wait on it
   // (for block j-1, by the softmax before a rescale and before the epilogue)
   // comes after P V of block j-3 has completed, so a parity wait is never
   // more than one phase behind
-  uint64_t* o_done = p_full + 2;
+  uint64_t* o_done = p_full + 4;
   uint64_t* fin = o_done + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   int* n_sel_slot = reinterpret_cast<int*>(smem + L::kMisc + 4);
@@ -108,7 +115,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     for (int t = 0; t < 2; ++t) {
       tc::mbar_init(s_full + 2 * t, 1);
       tc::mbar_init(s_full + 2 * t + 1, 1);
-      tc::mbar_init(p_full + t, 4);
+      tc::mbar_init(p_full + 2 * t, 4);
+      tc::mbar_init(p_full + 2 * t + 1, 4);
       tc::mbar_init(o_done + 2 * t, 1);
       tc::mbar_init(o_done + 2 * t + 1, 1);
     }
@@ -189,10 +197,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
       const uint32_t q_addr = tc::smem_u32(sQ), kv_addr = tc::smem_u32(sKV);
-      // Issue order: S_0(0) S_1(0) | S_0(j+1) S_1(j+1) PV_0(j) PV_1(j) | ...  S of
-      // the next block goes into the other buffer of its tile (free once
-      // P V of block j-1 has completed), so it is ready when the softmax of
-      // block j finishes.
       auto issue_s = [&](int t, int j) {
         const uint32_t k_addr = kv_addr + (j % kSpTcStages) * 2 * L::kKV;
 #pragma unroll
@@ -214,6 +218,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         }
         tc::mma_commit(o_done + 2 * t + (j & 1));
       };
+      // Issue order: S_0(0) S_1(0) | S_0(j+1) S_1(j+1) PV_0(j) PV_1(j) | ...  S of
+      // the next block goes into the other buffer of its tile, so it is
+      // ready when the softmax of block j finishes.
       bool ok = tc::mbar_wait(q_full, 0) && tc::mbar_wait(kv_full, 0);
       if (ok) {
         tc::tc_fence_after();
@@ -231,7 +238,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
           for (int t = 0; t < 2; ++t) issue_s(t, j + 1);
         }
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = tc::mbar_wait(p_full + t, j & 1))) break;
+          if (!(ok = tc::mbar_wait(p_full + 2 * t + (j & 1), (j >> 1) & 1))) break;
           tc::tc_fence_after();
           issue_pv(t, j);
         }
@@ -322,7 +329,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       tc::tmem_wait_st();
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(p_full + t);
+      if (lane == 0) tc::mbar_arrive(p_full + 2 * t + (j & 1));
     }
     // epilogue: out = sigmoid(gate) * O / l
     if (ok)
