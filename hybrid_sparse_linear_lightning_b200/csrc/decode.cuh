@@ -61,22 +61,19 @@ constexpr int kDecMaxLayers = 8;
 __host__ __device__ constexpr long long dec_key_stride(long long capb) { return (capb + 3) / 4 * 4; }
 
 // Control words at the start of the workspace (zeroed by the host before
-// each launch), each on its own 128-byte line: the barriers' arrival counts
-// and release flags, the P0 work counter, and per (batch, kv head) the
-// number of scored chunks.
+// each launch), each on its own 128-byte line: the barriers' arrival counts,
+// the work counters of P0 and P1, and per (batch, kv head) the number of
+// scored chunks.
 constexpr int kDecCtlBarriers = 2;
 constexpr int kDecLine = 32;            // words per 128-byte line
-__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (2 * kDecCtlBarriers + 2 + bg); }
+__host__ __device__ constexpr int dec_ctl_words(int bg) { return kDecLine * (kDecCtlBarriers + 2 + bg); }
 __device__ __forceinline__ unsigned* dec_bar_count(unsigned* ctl, int i) { return ctl + kDecLine * i; }
-__device__ __forceinline__ unsigned* dec_bar_flag(unsigned* ctl, int i) {
-  return ctl + kDecLine * (kDecCtlBarriers + i);
-}
 // work counters of P0 (phase 0) and P1 (phase 1)
 __device__ __forceinline__ unsigned* dec_work(unsigned* ctl, int phase) {
-  return ctl + kDecLine * (2 * kDecCtlBarriers + phase);
+  return ctl + kDecLine * (kDecCtlBarriers + phase);
 }
 __device__ __forceinline__ unsigned* dec_bg_done(unsigned* ctl, int bg) {
-  return ctl + kDecLine * (2 * kDecCtlBarriers + 2 + bg);
+  return ctl + kDecLine * (kDecCtlBarriers + 2 + bg);
 }
 
 // Persistent loop over `n` units in order: CTA x takes unit x first, and
@@ -152,32 +149,26 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
-// Grid barrier of a cooperative launch, bounded like every wait here.  The
-// last CTA to arrive runs `last` (whole CTA) before releasing the others.
-// Returns false (and sets the timeout bit) if the release did not come.
-template <typename F>
-__device__ __forceinline__ bool dec_grid_sync(unsigned* count, unsigned* flag, F last) {
-  __shared__ int s_last, s_ok;
+// Atomic add with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel_u32(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Grid barrier of a cooperative launch, bounded like every wait here.  Each
+// CTA arrives with one acquire-release add (after a CTA barrier, so it
+// releases everything the CTA wrote) and polls the count with acquire loads
+// until every CTA has arrived; the count is zeroed before the launch.
+// Returns false (and sets the timeout bit) if the others did not arrive.
+__device__ __forceinline__ bool dec_grid_sync(unsigned* count) {
+  __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(count, 1u) == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    last();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      atomicExch(flag, 1u);
-      s_ok = 1;
-    }
-  } else if (threadIdx.x == 0) {
     s_ok = 1;
-    if (ld_acquire_u32(flag) == 0u) {
+    if (atom_add_acq_rel_u32(count, 1u) + 1u < gridDim.x) {
       const long long t0 = clock64();
-      while (ld_acquire_u32(flag) == 0u) {
+      while (ld_acquire_u32(count) < gridDim.x) {
         if (clock64() - t0 > (1ll << 31)) {
           set_status(kStatusTimeout);
           s_ok = 0;
@@ -185,7 +176,6 @@ __device__ __forceinline__ bool dec_grid_sync(unsigned* count, unsigned* flag, F
         }
       }
     }
-    __threadfence();
   }
   __syncthreads();
   return s_ok != 0;
@@ -294,15 +284,10 @@ __device__ void dec_score_unit(const DecodeParams& p, int u, float* sm) {
   // the CTA that finishes the last chunk of (b, g) selects for it
   __shared__ int s_last_chunk;
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    s_last_chunk = atomicAdd(dec_bg_done(p.ctl, bg), 1u) == (unsigned)(p.n_chunks - 1);
-  }
+  if (tid == 0)   // releases this CTA's keys and bins; the last one acquires all the others'
+    s_last_chunk = atom_add_acq_rel_u32(dec_bg_done(p.ctl, bg), 1u) == (unsigned)(p.n_chunks - 1);
   __syncthreads();
-  if (s_last_chunk) {
-    __threadfence();
-    dec_select_bg<D>(p, bg, reinterpret_cast<unsigned char*>(sm));
-  }
+  if (s_last_chunk) dec_select_bg<D>(p, bg, reinterpret_cast<unsigned char*>(sm));
 }
 
 // One linear (layer, batch, head): S <- lam S + k^T v over the whole d x d
@@ -934,14 +919,14 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
     else if (u < n_score + p.B + n_direct) dec_direct_row(p, u - n_score - p.B);
     else dec_linear_unit<T, D>(p, u - n_score - p.B - n_direct, sm);
   });
-  if (!dec_grid_sync(dec_bar_count(p.ctl, 0), dec_bar_flag(p.ctl, 0), [] {})) return;
+  if (!dec_grid_sync(dec_bar_count(p.ctl, 0))) return;
   // P1: attention partials
   const int n_att = BG * p.width;
   if (p.Hq / p.Hkv <= 16)
     dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit_mma<D>(p, u, dec_smem); });
   else
     dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit<D>(p, u, dec_smem); });
-  if (!dec_grid_sync(dec_bar_count(p.ctl, 1), dec_bar_flag(p.ctl, 1), [] {})) return;
+  if (!dec_grid_sync(dec_bar_count(p.ctl, 1))) return;
   // P2: combine and gate
   for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {
     dec_combine_unit<T, D>(p, u, sm);
