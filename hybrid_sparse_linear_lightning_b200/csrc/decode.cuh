@@ -825,33 +825,37 @@ __device__ void dec_attn_unit_mma(const DecodeParams& p, int u, unsigned char* s
 }
 
 // Combine of the `width` partials of q head hq of batch b and the output
-// gate.  Thread (quarter of the partials, column).
+// gate, for value columns [32 cu, 32 cu + 32) (a head is split over D / 32
+// units so that more CTAs share the reads).  Warp w takes partials w, w + 16,
+// ...; lane l column 32 cu + l.
+constexpr int kDecCombCols = 32;
 template <typename T, int D>
 __device__ void dec_combine_unit(const DecodeParams& p, int u, float* sm) {
   constexpr int DP = D + 4;
-  constexpr int NQ = kDecThreads / D;
-  constexpr int kBatch = 18;             // partials in flight per thread
-  const int hq = u % p.Hq, b = u / p.Hq;
+  constexpr int NCU = D / kDecCombCols;          // units per head
+  constexpr int NG = kDecThreads / kDecCombCols; // partial groups (one per warp)
+  constexpr int kBatch = 8;                      // partials in flight per thread
+  const int cu = u % NCU, hq = (u / NCU) % p.Hq, b = u / (NCU * p.Hq);
   const int G = p.Hq / p.Hkv, g = hq / G, h = hq % G;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, grp = tid >> 5;
   float* wts = sm;                       // [width] weights, then [width] sums
   float* lsum = sm + p.width;
-  float* red = sm + 2 * p.width;         // [NQ][D]
+  float* red = sm + 2 * p.width;         // [NG][32]
   __shared__ float s_l;
   const float* pb = p.part + (((long long)b * p.Hkv + g) * p.width * G + h) * DP;
   const long long pstride = (long long)G * DP;
-  const int col = tid % D, qtr = tid / D;
-  float o = 0.f;
-  // this thread's first batch of partial columns is loaded before the weights
-  // are formed (every thread runs this block: it holds the CTA barriers)
+  const int col = cu * kDecCombCols + lane;
+  // this thread's first batch of partial columns and the gate are loaded
+  // before the weights are formed (every thread runs this block: it holds
+  // the CTA barriers)
   float pv[kBatch];
 #pragma unroll
   for (int v = 0; v < kBatch; ++v) {
-    const int e = qtr + v * NQ;
+    const int e = grp + v * NG;
     pv[v] = e < p.width ? __ldcg(pb + e * pstride + 4 + col) : 0.f;
   }
-  const long long off = ((long long)b * p.Hq + hq) * D + tid;
-  const float gt = tid < D ? ldf<T>(p.gate, off) : 0.f;     // the gate, loaded up front
+  const long long off = ((long long)b * p.Hq + hq) * D + col;
+  const float gt = tid < kDecCombCols ? ldf<T>(p.gate, off) : 0.f;
   for (int e = tid; e < p.width; e += kDecThreads) {
     wts[e] = __ldcg(pb + e * pstride);
     lsum[e] = __ldcg(pb + e * pstride + 1);
@@ -872,25 +876,26 @@ __device__ void dec_combine_unit(const DecodeParams& p, int u, float* sm) {
     if (tid == 0) s_l = L;
   }
   __syncthreads();
-  for (int e0 = qtr;; e0 += kBatch * NQ) {
+  float o = 0.f;
+  for (int e0 = grp;; e0 += kBatch * NG) {
 #pragma unroll
     for (int v = 0; v < kBatch; ++v) {
-      const int e = e0 + v * NQ;
+      const int e = e0 + v * NG;
       if (e < p.width) o = fmaf(wts[e], pv[v], o);
     }
-    if (e0 + kBatch * NQ >= p.width) break;
+    if (e0 + kBatch * NG >= p.width) break;
 #pragma unroll
     for (int v = 0; v < kBatch; ++v) {
-      const int e = e0 + kBatch * NQ + v * NQ;
+      const int e = e0 + kBatch * NG + v * NG;
       pv[v] = e < p.width ? __ldcg(pb + e * pstride + 4 + col) : 0.f;
     }
   }
-  red[qtr * D + col] = o;
+  red[grp * kDecCombCols + lane] = o;
   __syncthreads();
-  if (tid < D) {
+  if (tid < kDecCombCols) {
     float acc = 0.f;
 #pragma unroll
-    for (int r = 0; r < NQ; ++r) acc += red[r * D + tid];
+    for (int r = 0; r < NG; ++r) acc += red[r * kDecCombCols + tid];
     const float inv = s_l > 0.f ? 1.f / s_l : 0.f;
     static_cast<T*>(p.out)[off] = from_f32<T>(sigmoidf_(gt) * acc * inv);
   }
@@ -928,7 +933,7 @@ decode_step_kernel(const __grid_constant__ DecodeParams p) {
     dec_unit_loop(dec_work(p.ctl, 1), n_att, [&](int u) { dec_attn_unit<D>(p, u, dec_smem); });
   if (!dec_grid_sync(dec_bar_count(p.ctl, 1))) return;
   // P2: combine and gate
-  for (int u = blockIdx.x; u < p.B * p.Hq; u += gridDim.x) {
+  for (int u = blockIdx.x; u < p.B * p.Hq * (D / kDecCombCols); u += gridDim.x) {
     dec_combine_unit<T, D>(p, u, sm);
     __syncthreads();
   }
@@ -945,7 +950,7 @@ inline size_t decode_smem_bytes(int D, int G, int topk, long long kstride, int w
             (size_t)2 * G * D * 4 + (size_t)G * 8;                        // dec_attn_unit
   const size_t resolve = (size_t)2 * topk * 4 + 16 +
                          (size_t)kDecBndMax * 8 + (size_t)kstride * 4;   // dec_select_bg
-  const size_t comb = (size_t)2 * width * 4 + (size_t)(kDecThreads / D) * D * 4;
+  const size_t comb = (size_t)2 * width * 4 + (size_t)kDecThreads * 4;
   return std::max(std::max(std::max(score, lin), std::max(attn, resolve)), comb);
 }
 
