@@ -348,14 +348,14 @@ linear_segscan_kernel(const float* __restrict__ lambda, const float* __restrict_
   const float lam_last = (float)pow(lam, (double)(N - (n_seg - 1) * seg_len));
   float S = state_in ? state_in[i] : 0.f;
   float* p = seg_state + bh * n_seg * DD + e;
-  // segment sums are read 8 at a time so that the loads overlap
-  for (int s0 = 0; s0 < n_seg; s0 += 8) {
-    float ds[8];
+  // segment sums are read 16 at a time so that the loads overlap
+  for (int s0 = 0; s0 < n_seg; s0 += 16) {
+    float ds[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < 16; ++u)
       if (s0 + u < n_seg) ds[u] = p[(long long)(s0 + u) * DD];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int s = s0 + u;
       if (s < n_seg) {
         p[(long long)s * DD] = S;                   // state entering segment s
